@@ -1,0 +1,196 @@
+"""Attention oracle (CPU, double precision) — TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The CUDA library never calls it and
+shares no code with it; this module only marshals arguments to the plain C
+implementation in ``attn_oracle.c`` (built with gcc + OpenMP on first use).
+
+Functions cite the passages they follow in ``attn_oracle.c``.  In short:
+``attn_fwd`` is the plain definition softmax(mask(QK^T * scale)) V with a
+two-pass softmax over each materialised score row ("FlashAttention 2 原理与
+PyTorch 实战", sections 一 and 3.2); ``mask`` is the mask_mod predicate
+("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", sections 1 and 3);
+``decode_partials`` and ``combine`` are the split-KV decode written out as
+chunk-then-merge (same page, section 1).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_BUILD = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD, "liboracle_attn.so")
+_lock = threading.Lock()
+_lib = None
+
+_MASKS = {"none": 0, "causal": 1, "draft": 2}
+
+
+def build(force: bool = False) -> str:
+    """Compile ``attn_oracle.c`` into ``_build/liboracle_attn.so`` (gcc, -O2, OpenMP)."""
+    os.makedirs(_BUILD, exist_ok=True)
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-Wall", "-Wextra",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+            lib.oracle_mask.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, P]
+            lib.oracle_mask.restype = i32
+            lib.oracle_count_pairs.argtypes = [i32, i32, i32, i32, i32, i32, i32, P, P, i32]
+            lib.oracle_count_pairs.restype = i64
+            lib.oracle_attn_rows.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, i32, i32,
+                                             i32, i32, P, P, P, i64, P, P, i32]
+            lib.oracle_attn_rows.restype = i32
+            lib.oracle_decode_partials.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64,
+                                                   i32, i32, P, P, i32]
+            lib.oracle_decode_partials.restype = i32
+            lib.oracle_combine.argtypes = [P, P, i32, i64, i32, P, P]
+            lib.oracle_combine.restype = i32
+            lib.oracle_max_threads.argtypes = []
+            lib.oracle_max_threads.restype = i32
+            _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _bf16_bits(x) -> np.ndarray:
+    """bf16 tensor (torch) or uint16 array -> contiguous uint16 numpy array of the bits."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("oracle expects bf16 bit patterns as uint16")
+        return np.ascontiguousarray(x)
+    import torch
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"oracle expects bf16 inputs, got {x.dtype}")
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def _i32(x):
+    if x is None:
+        return None
+    if not isinstance(x, np.ndarray):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.int32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _mask_code(mask):
+    return mask if isinstance(mask, int) else _MASKS[mask]
+
+
+def mask(B, Lq, Lk, *, mask="none", window=(-1, -1), draft_block=1, doc_ids=None,
+         kv_lens=None) -> np.ndarray:
+    """Boolean mask [B, Lq, Lk]: entry (b, i, j) is True iff key j is visible to query row i."""
+    out = np.zeros((B, Lq, Lk), dtype=np.uint8)
+    doc = _i32(doc_ids)
+    kl = _i32(kv_lens)
+    rc = _load().oracle_mask(B, Lq, Lk, _mask_code(mask), int(window[0]), int(window[1]),
+                             int(draft_block), _ptr(doc), _ptr(kl), _ptr(out))
+    if rc:
+        raise ValueError("oracle_mask: invalid arguments")
+    return out.astype(bool)
+
+
+def count_pairs(B, Lq, Lk, *, mask="none", window=(-1, -1), draft_block=1, doc_ids=None,
+                kv_lens=None, nthreads=None) -> int:
+    """Allowed (query row, key) pairs summed over the batch, for ONE head."""
+    doc = _i32(doc_ids)
+    kl = _i32(kv_lens)
+    n = _load().oracle_count_pairs(B, Lq, Lk, _mask_code(mask), int(window[0]), int(window[1]),
+                                   int(draft_block), _ptr(doc), _ptr(kl),
+                                   int(nthreads or max_threads()))
+    if n < 0:
+        raise ValueError("oracle_count_pairs: invalid arguments")
+    return int(n)
+
+
+def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
+             doc_ids=None, kv_lens=None, rows=None, nthreads=None):
+    """Dense masked attention in double.
+
+    q: [B, Hq, Lq, d] bf16; k, v: [B, Hkv, Lk, d] bf16.  Returns (O, LSE) as
+    float64 numpy arrays, shaped [B, Hq, Lq, d] / [B, Hq, Lq], or [n, d] / [n]
+    when ``rows`` (flat indices (b*Hq + hq)*Lq + i) is given.
+    """
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    B, Hq, Lq, d = qb.shape
+    Bk, Hkv, Lk, dk = kb.shape
+    if vb.shape != kb.shape or Bk != B or dk != d:
+        raise ValueError("shape mismatch between q, k, v")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    doc = _i32(doc_ids)
+    kl = _i32(kv_lens)
+    if rows is not None:
+        rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64).reshape(-1))
+        n = rows.size
+    else:
+        n = B * Hq * Lq
+    o = np.zeros((n, d), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    rc = _load().oracle_attn_rows(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Lq, Lk, d,
+                                  float(scale), _mask_code(mask), int(window[0]), int(window[1]),
+                                  int(draft_block), _ptr(doc), _ptr(kl), _ptr(rows), n,
+                                  _ptr(o), _ptr(lse), int(nthreads or max_threads()))
+    if rc:
+        raise ValueError(f"oracle_attn_rows failed ({rc})")
+    if rows is None:
+        return o.reshape(B, Hq, Lq, d), lse.reshape(B, Hq, Lq)
+    return o, lse
+
+
+def decode_partials(q, k, v, kv_lens, *, chunk, nsplit=None, scale=None, nthreads=None):
+    """Per-chunk partial (O_s, LSE_s) of the split-KV decode; shapes [S, B*Hq*Lq, d] / [S, B*Hq*Lq]."""
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    B, Hq, Lq, d = qb.shape
+    _, Hkv, Lk, _ = kb.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    if nsplit is None:
+        nsplit = max(1, -(-Lk // chunk))
+    kl = _i32(kv_lens)
+    nrows = B * Hq * Lq
+    o = np.zeros((nsplit, nrows, d), dtype=np.float64)
+    lse = np.zeros((nsplit, nrows), dtype=np.float64)
+    rc = _load().oracle_decode_partials(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(kl), B, Hq, Hkv, Lq,
+                                        Lk, d, float(scale), int(chunk), int(nsplit), _ptr(o),
+                                        _ptr(lse), int(nthreads or max_threads()))
+    if rc:
+        raise ValueError(f"oracle_decode_partials failed ({rc})")
+    return o, lse
+
+
+def combine(o_part, lse_part):
+    """LSE-weighted merge of split partials: ([S, n, d], [S, n]) -> ([n, d], [n])."""
+    o_part = np.ascontiguousarray(o_part, dtype=np.float64)
+    lse_part = np.ascontiguousarray(lse_part, dtype=np.float64)
+    S, n, d = o_part.shape
+    o = np.zeros((n, d), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    rc = _load().oracle_combine(_ptr(o_part), _ptr(lse_part), S, n, d, _ptr(o), _ptr(lse))
+    if rc:
+        raise ValueError("oracle_combine failed")
+    return o, lse

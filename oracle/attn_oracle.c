@@ -1,0 +1,357 @@
+/*
+ * Attention oracle: plain, slow, obviously correct CPU attention in double.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the bench's
+ * CPU-baseline leg may call this code.  It shares nothing with the CUDA path
+ * (no headers, helpers, tables or constants) and the CUDA path never calls it.
+ *
+ * What it computes (plain definition; the tiled GPU method reaches the same
+ * result up to rounding order):
+ *
+ *   S = scale * Q K^T, masked entries set aside, P = softmax(S) row-wise,
+ *   O = P V, LSE = log sum_j exp(S_ij) over the allowed j (natural log).
+ *
+ *   - "FlashAttention 2 原理与 PyTorch 实战", section 一 (the memory bottleneck):
+ *     the standard formula softmax(QK^T / sqrt(d)) V, computed as S, then
+ *     P = softmax(S), then O = P V.  Here S is materialised one query row at a
+ *     time (the row's scores, then a max pass, then a sum pass).
+ *   - same page, section 3.2 (online softmax): the running max M and sum L;
+ *     the oracle does the plain two-pass softmax the online form reproduces.
+ *   - "FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", section 1: a mask is a
+ *     predicate mask_mod(b, h, q_idx, kv_idx) -> bool (causal, sliding window,
+ *     non-causal, document mask); section 3 (finding 1): the causal window
+ *     (w, 0) is made symmetric (w, w) so bidirectional draft queries look both
+ *     ways; the block-diffusion draft mask lets a draft token see the context
+ *     and every token of its own block.
+ *
+ * Readings taken where the pages are silent (each is also listed in the
+ * design notes):
+ *   - query row i sits at absolute position p = Lk_b - Lq + i (bottom-right
+ *     alignment), where Lk_b = kv_lens[b] when given, else Lk;
+ *   - window bounds are inclusive: p - w_left <= j <= p + w_right; -1 means
+ *     that side is unbounded;
+ *   - the draft-block mask allows j iff floor(j / Bd) <= floor(p / Bd)
+ *     (own block bidirectionally, every earlier block, no later block);
+ *     causal is the case Bd = 1;
+ *   - the document mask allows j iff doc[b][j] == doc[b][p]; it needs p >= 0;
+ *   - the mask terms combine by logical AND, with j < Lk_b always required;
+ *   - a row with no allowed key gets O = 0 and LSE = -inf;
+ *   - GQA maps query head hq to KV head hq / (Hq / Hkv);
+ *   - LSE is the natural log of the sum of exp of the scaled scores.
+ *
+ * Inputs are the bf16 bit patterns the GPU receives, widened exactly to
+ * double.  Layout: contiguous [B, H, L, D] for Q, K, V and O; [B, H, L] for
+ * LSE; [B, Lk] int32 for document ids; [B] int32 for KV lengths.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_MASK_NONE 0
+#define ORACLE_MASK_CAUSAL 1
+#define ORACLE_MASK_DRAFT_BLOCK 2
+
+static double bf16_bits_to_double(uint16_t h) {
+  uint32_t u = ((uint32_t)h) << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Floor division for a possibly negative numerator, positive divisor. */
+static int64_t floor_div(int64_t a, int64_t b) {
+  int64_t q = a / b;
+  if ((a % b) != 0 && (a < 0)) q -= 1;
+  return q;
+}
+
+typedef struct {
+  int B, Lq, Lk;
+  int mask_kind;
+  int window_l, window_r;
+  int draft_block;
+  const int32_t* doc_ids; /* [B, Lk] or NULL */
+  const int32_t* kv_lens; /* [B] or NULL */
+} mask_spec;
+
+static int key_count(const mask_spec* m, int b) {
+  return m->kv_lens ? m->kv_lens[b] : m->Lk;
+}
+
+/* mask_mod(b, q_idx = i, kv_idx = j): is key j visible to query row i? */
+static int allowed(const mask_spec* m, int b, int i, int j) {
+  int64_t lk_b = key_count(m, b);
+  if (j < 0 || j >= lk_b) return 0;
+  int64_t p = lk_b - m->Lq + i; /* absolute position of query row i */
+  switch (m->mask_kind) {
+    case ORACLE_MASK_NONE:
+      break;
+    case ORACLE_MASK_CAUSAL:
+      if (!(j <= p)) return 0;
+      break;
+    case ORACLE_MASK_DRAFT_BLOCK:
+      if (!(floor_div(j, m->draft_block) <= floor_div(p, m->draft_block))) return 0;
+      break;
+    default:
+      return 0;
+  }
+  if (m->window_l >= 0 && !(j >= p - m->window_l)) return 0;
+  if (m->window_r >= 0 && !(j <= p + m->window_r)) return 0;
+  if (m->doc_ids) {
+    if (p < 0 || p >= m->Lk) return 0;
+    const int32_t* doc = m->doc_ids + (int64_t)b * m->Lk;
+    if (doc[j] != doc[p]) return 0;
+  }
+  return 1;
+}
+
+static int check_mask_spec(const mask_spec* m) {
+  if (m->B < 0 || m->Lq < 0 || m->Lk < 0) return -1;
+  if (m->mask_kind < 0 || m->mask_kind > 2) return -1;
+  if (m->mask_kind == ORACLE_MASK_DRAFT_BLOCK && m->draft_block < 1) return -1;
+  if (m->window_l < -1 || m->window_r < -1) return -1;
+  if (m->kv_lens) {
+    for (int b = 0; b < m->B; ++b)
+      if (m->kv_lens[b] < 0 || m->kv_lens[b] > m->Lk) return -1;
+  }
+  return 0;
+}
+
+/* The boolean mask, one byte per (b, i, j): out is [B, Lq, Lk]. */
+int oracle_mask(int B, int Lq, int Lk, int mask_kind, int window_l, int window_r,
+                int draft_block, const int32_t* doc_ids, const int32_t* kv_lens,
+                uint8_t* out) {
+  mask_spec m = {B, Lq, Lk, mask_kind, window_l, window_r, draft_block, doc_ids, kv_lens};
+  if (check_mask_spec(&m)) return -1;
+  for (int b = 0; b < B; ++b)
+    for (int i = 0; i < Lq; ++i)
+      for (int j = 0; j < Lk; ++j)
+        out[((int64_t)b * Lq + i) * Lk + j] = (uint8_t)allowed(&m, b, i, j);
+  return 0;
+}
+
+/* Number of allowed (i, j) pairs summed over the batch (one head's worth).
+   Multiply by Hq for the whole call. */
+int64_t oracle_count_pairs(int B, int Lq, int Lk, int mask_kind, int window_l, int window_r,
+                           int draft_block, const int32_t* doc_ids, const int32_t* kv_lens,
+                           int nthreads) {
+  mask_spec m = {B, Lq, Lk, mask_kind, window_l, window_r, draft_block, doc_ids, kv_lens};
+  if (check_mask_spec(&m)) return -1;
+  int64_t total = 0;
+  int64_t nrows = (int64_t)B * Lq;
+#pragma omp parallel for schedule(dynamic, 64) reduction(+ : total) num_threads(nthreads)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int b = (int)(r / Lq), i = (int)(r % Lq);
+    int64_t c = 0;
+    for (int j = 0; j < Lk; ++j) c += allowed(&m, b, i, j);
+    total += c;
+  }
+  return total;
+}
+
+/*
+ * One query row over the keys [j_lo, j_hi) that the mask allows:
+ * scores, max pass, sum pass, weighted sum of V.  Writes d values to o_row
+ * and returns the row's LSE (-inf when no key is allowed; o_row is then 0).
+ */
+static double attend_row(const uint16_t* q_row, const uint16_t* k_head, const uint16_t* v_head,
+                         int d, double scale, const mask_spec* m, int b, int i, int j_lo,
+                         int j_hi, double* s_buf, uint8_t* ok_buf, double* q_buf,
+                         double* o_row) {
+  for (int c = 0; c < d; ++c) q_buf[c] = bf16_bits_to_double(q_row[c]);
+  /* scores of the row: S_ij = scale * sum_c Q_ic K_jc */
+  int any = 0;
+  for (int j = j_lo; j < j_hi; ++j) {
+    ok_buf[j - j_lo] = (uint8_t)allowed(m, b, i, j);
+    if (!ok_buf[j - j_lo]) continue;
+    const uint16_t* k_row = k_head + (int64_t)j * d;
+    double acc = 0.0;
+    for (int c = 0; c < d; ++c) acc += q_buf[c] * bf16_bits_to_double(k_row[c]);
+    s_buf[j - j_lo] = scale * acc;
+    any = 1;
+  }
+  for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+  if (!any) return -INFINITY;
+  /* pass 1: row max */
+  double mx = -INFINITY;
+  for (int j = j_lo; j < j_hi; ++j)
+    if (ok_buf[j - j_lo] && s_buf[j - j_lo] > mx) mx = s_buf[j - j_lo];
+  /* pass 2: sum of exp(s - max) */
+  double l = 0.0;
+  for (int j = j_lo; j < j_hi; ++j)
+    if (ok_buf[j - j_lo]) l += exp(s_buf[j - j_lo] - mx);
+  /* O = sum_j P_ij V_j with P_ij = exp(s_ij - max) / l */
+  for (int j = j_lo; j < j_hi; ++j) {
+    if (!ok_buf[j - j_lo]) continue;
+    double p = exp(s_buf[j - j_lo] - mx) / l;
+    const uint16_t* v_row = v_head + (int64_t)j * d;
+    for (int c = 0; c < d; ++c) o_row[c] += p * bf16_bits_to_double(v_row[c]);
+  }
+  return mx + log(l);
+}
+
+static int check_shapes(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Lq < 0 || Lk < 0 || d < 1) return -1;
+  if (Hq % Hkv) return -1;
+  return 0;
+}
+
+/*
+ * Attention over selected rows.  rows[r] is a flat row index
+ * (b * Hq + hq) * Lq + i; rows == NULL means every row in order.
+ * o is [nrows, d], lse is [nrows].
+ */
+int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                     int Hkv, int Lq, int Lk, int d, double scale, int mask_kind, int window_l,
+                     int window_r, int draft_block, const int32_t* doc_ids,
+                     const int32_t* kv_lens, const int64_t* rows, int64_t nrows, double* o,
+                     double* lse, int nthreads) {
+  if (check_shapes(B, Hq, Hkv, Lq, Lk, d)) return -1;
+  mask_spec m = {B, Lq, Lk, mask_kind, window_l, window_r, draft_block, doc_ids, kv_lens};
+  if (check_mask_spec(&m)) return -1;
+  int64_t total_rows = (int64_t)B * Hq * Lq;
+  if (!rows) nrows = total_rows;
+  for (int64_t r = 0; r < (rows ? nrows : 0); ++r)
+    if (rows[r] < 0 || rows[r] >= total_rows) return -1;
+  int group = Hq / Hkv;
+  int err = 0;
+#pragma omp parallel num_threads(nthreads)
+  {
+    double* s_buf = (double*)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+    uint8_t* ok_buf = (uint8_t*)malloc((size_t)(Lk > 0 ? Lk : 1));
+    double* q_buf = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!s_buf || !ok_buf || !q_buf) {
+#pragma omp atomic write
+      err = 1;
+    }
+#pragma omp for schedule(dynamic, 8)
+    for (int64_t r = 0; r < nrows; ++r) {
+      if (err) continue;
+      int64_t flat = rows ? rows[r] : r;
+      int i = (int)(flat % Lq);
+      int64_t bh = flat / Lq;
+      int hq = (int)(bh % Hq);
+      int b = (int)(bh / Hq);
+      int hkv = hq / group;
+      const uint16_t* q_row = q + flat * d;
+      const uint16_t* k_head = k + ((int64_t)b * Hkv + hkv) * Lk * d;
+      const uint16_t* v_head = v + ((int64_t)b * Hkv + hkv) * Lk * d;
+      lse[r] = attend_row(q_row, k_head, v_head, d, scale, &m, b, i, 0, Lk, s_buf, ok_buf,
+                          q_buf, o + r * d);
+    }
+    free(s_buf);
+    free(ok_buf);
+    free(q_buf);
+  }
+  return err ? -2 : 0;
+}
+
+/*
+ * Split-KV decode, step 1 (FlexDecoding / FlashDecoding style split-KV, "FlexAttention
+ * 是什么，以及 DFlash2 之谜的完整侦破", section 1): the keys of sequence b,
+ * [0, kv_lens[b]), are cut into chunks [s*chunk, (s+1)*chunk); split s attends
+ * over its own chunk only and yields a normalised partial output O_s and its
+ * LSE_s.  An empty chunk yields O_s = 0, LSE_s = -inf.
+ * o_part is [nsplit, B*Hq*Lq, d]; lse_part is [nsplit, B*Hq*Lq].
+ */
+int oracle_decode_partials(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq, int Lk,
+                           int d, double scale, int chunk, int nsplit, double* o_part,
+                           double* lse_part, int nthreads) {
+  if (check_shapes(B, Hq, Hkv, Lq, Lk, d) || chunk < 1 || nsplit < 1) return -1;
+  if (!kv_lens) return -1;
+  mask_spec m = {B, Lq, Lk, ORACLE_MASK_NONE, -1, -1, 1, NULL, kv_lens};
+  if (check_mask_spec(&m)) return -1;
+  if ((int64_t)nsplit * chunk < Lk) return -1;
+  int64_t nrows = (int64_t)B * Hq * Lq;
+  int group = Hq / Hkv;
+  int err = 0;
+#pragma omp parallel num_threads(nthreads)
+  {
+    double* s_buf = (double*)malloc(sizeof(double) * (size_t)chunk);
+    uint8_t* ok_buf = (uint8_t*)malloc((size_t)chunk);
+    double* q_buf = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!s_buf || !ok_buf || !q_buf) {
+#pragma omp atomic write
+      err = 1;
+    }
+#pragma omp for schedule(dynamic, 4) collapse(2)
+    for (int s = 0; s < nsplit; ++s) {
+      for (int64_t r = 0; r < nrows; ++r) {
+        if (err) continue;
+        int i = (int)(r % Lq);
+        int64_t bh = r / Lq;
+        int hq = (int)(bh % Hq);
+        int b = (int)(bh / Hq);
+        int hkv = hq / group;
+        int j_lo = s * chunk;
+        int j_hi = j_lo + chunk;
+        if (j_hi > kv_lens[b]) j_hi = kv_lens[b];
+        double* o_row = o_part + ((int64_t)s * nrows + r) * d;
+        if (j_lo >= j_hi) {
+          for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+          lse_part[(int64_t)s * nrows + r] = -INFINITY;
+          continue;
+        }
+        lse_part[(int64_t)s * nrows + r] =
+            attend_row(q + r * d, k + ((int64_t)b * Hkv + hkv) * Lk * d,
+                       v + ((int64_t)b * Hkv + hkv) * Lk * d, d, scale, &m, b, i, j_lo, j_hi,
+                       s_buf, ok_buf, q_buf, o_row);
+      }
+    }
+    free(s_buf);
+    free(ok_buf);
+    free(q_buf);
+  }
+  return err ? -2 : 0;
+}
+
+/*
+ * Split-KV decode, step 2: the LSE-weighted combine.
+ *   LSE = log sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s.
+ * Splits with LSE_s = -inf contribute nothing; if all are -inf the row is
+ * fully masked (O = 0, LSE = -inf).
+ */
+int oracle_combine(const double* o_part, const double* lse_part, int nsplit, int64_t nrows,
+                   int d, double* o, double* lse) {
+  if (nsplit < 1 || nrows < 0 || d < 1) return -1;
+  for (int64_t r = 0; r < nrows; ++r) {
+    double mx = -INFINITY;
+    for (int s = 0; s < nsplit; ++s)
+      if (lse_part[(int64_t)s * nrows + r] > mx) mx = lse_part[(int64_t)s * nrows + r];
+    double* o_row = o + r * d;
+    for (int c = 0; c < d; ++c) o_row[c] = 0.0;
+    if (mx == -INFINITY) {
+      lse[r] = -INFINITY;
+      continue;
+    }
+    double sum = 0.0;
+    for (int s = 0; s < nsplit; ++s) {
+      double ls = lse_part[(int64_t)s * nrows + r];
+      if (ls == -INFINITY) continue;
+      sum += exp(ls - mx);
+    }
+    double total = mx + log(sum);
+    for (int s = 0; s < nsplit; ++s) {
+      double ls = lse_part[(int64_t)s * nrows + r];
+      if (ls == -INFINITY) continue;
+      double w = exp(ls - total);
+      const double* os = o_part + ((int64_t)s * nrows + r) * d;
+      for (int c = 0; c < d; ++c) o_row[c] += w * os[c];
+    }
+    lse[r] = total;
+  }
+  return 0;
+}
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

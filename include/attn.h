@@ -1,0 +1,166 @@
+/*
+ * attn.h — C ABI of the B200 (sm_100a) fused attention forward library.
+ *
+ * The library computes O = softmax(mask(Q K^T * scale)) V and the per-row
+ * log-sum-exp with a fused, tiled kernel: each 128-row query tile streams
+ * 128-key K/V tiles through shared memory and keeps a running max and sum
+ * (online softmax), so the N x N score matrix never reaches device memory
+ * ("FlashAttention 2 原理与 PyTorch 实战", sections 一, 3.1 and 3.2).  A split-KV
+ * decode for short queries over a long cache, with GQA, and its LSE-weighted
+ * combine follow FlexDecoding / FlashDecoding ("FlexAttention 是什么，以及
+ * DFlash2 之谜的完整侦破", section 1).
+ *
+ * Conventions shared by every entry point
+ *   - Element type: bf16 for Q, K, V and O (no dtype argument; the pages'
+ *     kernels take bf16/fp16 only, "FlashAttention 2 原理与 PyTorch 实战",
+ *     section 七).  LSE is fp32, natural log.
+ *   - Layout: contiguous [B, H, L, D] (PyTorch's SDPA layout, same page,
+ *     section 二), i.e. element (b, h, l, c) at ((b*H + h)*L + l)*D + c.
+ *   - GQA: query head hq reads KV head hq / (Hq / Hkv).
+ *   - All pointers are DEVICE pointers owned by the caller; the library keeps
+ *     none of them after the call returns.  Q, K, V, O and the workspace must
+ *     be 16-byte aligned; LSE, doc_ids and kv_lens 4-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     enqueue work and return; they never synchronise the device and never
+ *     allocate device memory.
+ *   - Arguments are validated on the host before anything is launched; an
+ *     invalid call returns a status and enqueues nothing.  A launch failure
+ *     returns ATTN_ERR_CUDA.  Kernel-side problems (a bounded wait that ran
+ *     out, a kv_lens entry out of range) are recorded in a device error word
+ *     read by attn_get_device_error().
+ *   - Inputs must be finite, except the decode cache past kv_lens[b], which
+ *     may hold anything (it is never used, not even multiplied by zero).
+ */
+#ifndef ATTN_B200_ATTN_H_
+#define ATTN_B200_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape or mask argument */
+  ATTN_ERR_UNSUPPORTED = 2, /* valid request outside what is built (e.g. d not 64/128) */
+  ATTN_ERR_WORKSPACE = 3,   /* decode workspace missing or too small */
+  ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call or launch failed */
+  ATTN_ERR_TIMEOUT = 5      /* a kernel gave up on a bounded wait (device error word) */
+} attn_status_t;
+
+typedef enum {
+  ATTN_MASK_NONE = 0,       /* bidirectional */
+  ATTN_MASK_CAUSAL = 1,     /* key j visible iff j <= p */
+  ATTN_MASK_DRAFT_BLOCK = 2 /* key j visible iff floor(j/Bd) <= floor(p/Bd) */
+} attn_mask_kind_t;
+
+/*
+ * attn_fwd — prefill attention forward.
+ *
+ * Defines ("FlashAttention 2 原理与 PyTorch 实战", section 一; masks from
+ * "FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", sections 1 and 3):
+ *   for b < B, hq < Hq, query row i < Lq at absolute position p = Lk - Lq + i
+ *   (bottom-right alignment), key j < Lk is visible iff
+ *     base(p, j)                                     (per mask_kind above)
+ *     and (window_l < 0 or j >= p - window_l)        (sliding window, inclusive;
+ *     and (window_r < 0 or j <= p + window_r)         -1 = unbounded side)
+ *     and (doc_ids == NULL or doc_ids[b][j] == doc_ids[b][p]).
+ *   S_ij = scale * <Q[b,hq,i,:], K[b,hkv,j,:]> over visible j;
+ *   O[b,hq,i,:] = sum_j softmax_j(S_ij) V[b,hkv,j,:];  LSE[b,hq,i] = log sum_j exp(S_ij).
+ *   A row with no visible key gets O = 0 and LSE = -inf.
+ *   The block-diffusion draft mask with the symmetric window (w, w) is
+ *   mask_kind = ATTN_MASK_DRAFT_BLOCK, draft_block = Bd, window_l = window_r = w.
+ *
+ * Arguments
+ *   q        [B, Hq, Lq, d] bf16, read
+ *   k, v     [B, Hkv, Lk, d] bf16, read
+ *   o        [B, Hq, Lq, d] bf16, written
+ *   lse      [B, Hq, Lq] fp32, written
+ *   B, Hq, Hkv, Lq, Lk >= 1, Hq % Hkv == 0; d in {64, 128} (else UNSUPPORTED);
+ *   Lk <= 524288 (else UNSUPPORTED)
+ *   scale    > 0 and finite (1/sqrt(d) is the usual choice)
+ *   mask_kind  one of attn_mask_kind_t; window_l, window_r >= -1;
+ *   draft_block >= 1 (read only for ATTN_MASK_DRAFT_BLOCK)
+ *   doc_ids  [B, Lk] int32 or NULL; when given, Lq <= Lk is required
+ *   stream   cudaStream_t
+ * Errors: INVALID_ARG / UNSUPPORTED before any launch; CUDA on launch failure.
+ */
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_kind,
+                       int window_l, int window_r, int draft_block, const int32_t* doc_ids,
+                       void* stream);
+
+/*
+ * attn_decode_num_splits — how many KV splits attn_decode_splitkv uses.
+ *
+ * The keys [0, Lk_max) are cut into nsplit chunks of `chunk` keys each, a
+ * whole number of 128-key tiles; split s covers [s*chunk, (s+1)*chunk) and
+ * sequence b uses the first ceil(kv_lens[b] / chunk) splits.  num_splits > 0
+ * asks for that many chunks (capped at ceil(Lk_max / 128)); 0 lets the
+ * library choose from B * Hkv, Lk_max and the device's SM count.
+ * Returns the split count (>= 1) and stores the chunk length in *chunk_keys
+ * (nullable); returns -1 for invalid arguments.
+ */
+int attn_decode_num_splits(int B, int Hq, int Hkv, int Lq, int Lk_max, int d, int num_splits,
+                           int* chunk_keys);
+
+/*
+ * attn_decode_workspace_size — bytes of caller-owned device workspace that
+ * attn_decode_splitkv needs for the same arguments; 0 for invalid arguments.
+ *
+ * Workspace layout (documented so tests can read the partial results):
+ *   offset 0:           fp32 O_s  [nsplit, B*Hq*Lq, d]   (normalised per split)
+ *   offset ws_lse_off:  fp32 LSE_s [nsplit, B*Hq*Lq]
+ *   where ws_lse_off = round_up(nsplit*B*Hq*Lq*d*4, 256).
+ *   Rows of splits that hold no key of their sequence are not written.
+ */
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk_max, int d,
+                                  int num_splits);
+
+/*
+ * attn_decode_splitkv — split-KV decode attention (non-causal over the cache).
+ *
+ * Defines: for each b, query head hq and query row i < Lq, the keys visible
+ * are exactly [0, kv_lens[b]) of the cache; O and LSE as in attn_fwd with no
+ * mask.  Computed in two launches on `stream` ("FlexAttention 是什么，以及
+ * DFlash2 之谜的完整侦破", section 1: a short query over a long KV is split
+ * across CTAs, then merged): (1) per (b, kv head, split) a partial O_s and
+ * LSE_s over that chunk, for all Hq/Hkv query heads of the group at once;
+ * (2) the combine LSE = log sum_s exp(LSE_s), O = sum_s exp(LSE_s - LSE) O_s.
+ *
+ * Arguments
+ *   q        [B, Hq, Lq, d] bf16, read
+ *   k_cache, v_cache  [B, Hkv, Lk_max, d] bf16, read only below kv_lens[b]
+ *   o        [B, Hq, Lq, d] bf16, written;  lse [B, Hq, Lq] fp32, written
+ *   kv_lens  [B] int32 DEVICE array, each in [1, Lk_max]; an entry outside
+ *            [0, Lk_max] is clamped and flags the device error word
+ *   d in {64, 128}; scale > 0; num_splits as in attn_decode_num_splits
+ *   workspace, ws_bytes  caller-owned device buffer of at least
+ *            attn_decode_workspace_size(...) bytes (else ATTN_ERR_WORKSPACE)
+ * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch; CUDA on
+ * launch failure.
+ */
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                                  void* o, float* lse, const int32_t* kv_lens, int B, int Hq,
+                                  int Hkv, int Lq, int Lk_max, int d, float scale, int num_splits,
+                                  void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * attn_get_device_error — synchronise `stream`, then read and clear the
+ * device error word of the current device.  Returns ATTN_OK, ATTN_ERR_TIMEOUT
+ * (a kernel abandoned a bounded wait), ATTN_ERR_INVALID_ARG (a kv_lens entry
+ * was out of range) or ATTN_ERR_CUDA (the synchronisation itself failed).
+ * `raw_bits` (nullable) receives the raw error bits.
+ */
+attn_status_t attn_get_device_error(void* stream, int* raw_bits);
+
+/* Static, human-readable name of a status code. */
+const char* attn_status_string(attn_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_ATTN_H_ */

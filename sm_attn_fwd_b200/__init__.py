@@ -1,0 +1,201 @@
+"""Python binding of the B200 attention C ABI (``include/attn.h``).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library ``_lib/libattn_b200.so``.  PyTorch supplies device memory and the
+current stream.  There is no fallback path: if the library is missing or the
+tensors are not on a CUDA device, the calls raise.
+
+Entry points (same names as the C ABI):
+  attn_fwd(q, k, v, ...)                 -> (o, lse)
+  attn_decode_splitkv(q, k, v, kv_lens, ...) -> (o, lse)
+  attn_decode_num_splits(...), attn_decode_workspace_size(...)
+  attn_get_device_error(stream=None)     -> (status, raw_bits)
+  attn_status_string(status)             -> str
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "AttnError", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
+    "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
+    "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
+    "attn_fwd", "attn_decode_splitkv", "attn_decode_num_splits",
+    "attn_decode_workspace_size", "attn_get_device_error", "attn_status_string",
+    "EXPORTED_SYMBOLS",
+]
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_WORKSPACE = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_TIMEOUT = 5
+
+MASK_NONE = 0
+MASK_CAUSAL = 1
+MASK_DRAFT_BLOCK = 2
+_MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
+
+EXPORTED_SYMBOLS = (
+    "attn_fwd", "attn_decode_num_splits", "attn_decode_workspace_size",
+    "attn_decode_splitkv", "attn_get_device_error", "attn_status_string",
+)
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "_lib", "libattn_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {attn_status_string(status)}")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load the CUDA library (building it first if it is absent and nvcc exists)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            from . import build as _build
+            _build.build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, i32, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.attn_fwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, i32,
+                                 i32, P, P]
+        lib.attn_fwd.restype = i32
+        lib.attn_decode_num_splits.argtypes = [i32] * 7 + [ctypes.POINTER(ctypes.c_int)]
+        lib.attn_decode_num_splits.restype = i32
+        lib.attn_decode_workspace_size.argtypes = [i32] * 7
+        lib.attn_decode_workspace_size.restype = sz
+        lib.attn_decode_splitkv.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
+                                            i32, P, sz, P]
+        lib.attn_decode_splitkv.restype = i32
+        lib.attn_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
+        lib.attn_get_device_error.restype = i32
+        lib.attn_status_string.argtypes = [i32]
+        lib.attn_status_string.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def attn_status_string(status: int) -> str:
+    return load_library().attn_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_bf16(name, t):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+    if t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, H, L, D] tensor")
+
+
+def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
+             doc_ids=None, o=None, lse=None, stream=None):
+    """Prefill attention forward (see ``attn_fwd`` in include/attn.h).
+
+    q: [B, Hq, Lq, d], k/v: [B, Hkv, Lk, d], bf16 CUDA tensors.  Returns
+    (o bf16 [B, Hq, Lq, d], lse fp32 [B, Hq, Lq]).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_bf16(name, t)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    if doc_ids is not None:
+        if doc_ids.dtype != torch.int32 or not doc_ids.is_cuda or not doc_ids.is_contiguous():
+            raise ValueError("doc_ids must be a contiguous int32 CUDA tensor [B, Lk]")
+    mk = mask if isinstance(mask, int) else _MASKS[mask]
+    st = load_library().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq,
+                                 Lk, d, float(scale), mk, int(window[0]), int(window[1]),
+                                 int(draft_block), _ptr(doc_ids), _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def attn_decode_num_splits(B, Hq, Hkv, Lq, Lk_max, d, num_splits=0):
+    """(nsplit, chunk_keys) that attn_decode_splitkv uses for these arguments."""
+    chunk = ctypes.c_int(0)
+    n = load_library().attn_decode_num_splits(B, Hq, Hkv, Lq, Lk_max, d, num_splits,
+                                              ctypes.byref(chunk))
+    if n < 0:
+        raise AttnError(ATTN_ERR_INVALID_ARG, "attn_decode_num_splits")
+    return int(n), int(chunk.value)
+
+
+def attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk_max, d, num_splits=0) -> int:
+    n = load_library().attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk_max, d, num_splits)
+    if n == 0:
+        raise AttnError(ATTN_ERR_INVALID_ARG, "attn_decode_workspace_size")
+    return int(n)
+
+
+def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, *, scale=None, num_splits=0,
+                        workspace=None, o=None, lse=None, stream=None):
+    """Split-KV decode (see ``attn_decode_splitkv`` in include/attn.h).
+
+    q: [B, Hq, Lq, d]; k_cache/v_cache: [B, Hkv, Lk_max, d]; kv_lens: int32 [B]
+    on the device.  ``workspace`` (uint8 CUDA tensor) is allocated here when
+    not given.  Returns (o, lse).
+    """
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_bf16(name, t)
+    if kv_lens.dtype != torch.int32 or not kv_lens.is_cuda or not kv_lens.is_contiguous():
+        raise ValueError("kv_lens must be a contiguous int32 CUDA tensor [B]")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk_max, _ = k_cache.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk_max, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_decode_splitkv(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), _ptr(kv_lens), B, Hq, Hkv,
+        Lq, Lk_max, d, float(scale), int(num_splits), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_get_device_error(stream=None):
+    """Synchronise the stream and read/clear the device error word: (status, raw_bits)."""
+    bits = ctypes.c_int(0)
+    dev = torch.cuda.current_device()
+    st = load_library().attn_get_device_error(_stream_handle(stream, dev), ctypes.byref(bits))
+    return int(st), int(bits.value)

@@ -1,0 +1,280 @@
+// Host side of the C ABI declared in include/attn.h: argument validation,
+// split planning, TMA tensor-map encoding and kernel launches.  Nothing here
+// allocates device memory or synchronises, except attn_get_device_error.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_params.h"
+
+namespace attn {
+template <int D, bool kDecode>
+cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                       const FwdParams&, dim3, cudaStream_t);
+template <int D>
+cudaError_t launch_combine(const FwdParams&, cudaStream_t);
+int* device_error_word();
+}  // namespace attn
+
+namespace {
+
+using attn::FwdParams;
+using attn::kBlockM;
+using attn::kBlockN;
+
+constexpr long long kMaxGridY = 65535;
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// bf16 tensor map of rank 2 or 3 (innermost first), 64 x 128 boxes, 128-byte
+// swizzle; out-of-range rows read as zero.
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3];
+  cuuint64_t gstride[2];
+  cuuint32_t box[3] = {64, (cuuint32_t)kBlockN, 1};
+  cuuint32_t estride[3] = {1, 1, 1};
+  uint64_t stride = 2;
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    if (i > 0) gstride[i - 1] = stride;
+    stride *= dims[i];
+  }
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
+                  gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      n = v;
+  }
+  return n;
+}
+
+long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+struct SplitPlan {
+  int nsplit;
+  int chunk;
+  int row_tiles;
+};
+
+// Returns false for invalid shape arguments.
+bool plan_splits(int B, int Hq, int Hkv, int Lq, int Lk_max, int d, int num_splits,
+                 SplitPlan* plan) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk_max < 1 || d < 1 || num_splits < 0) return false;
+  if (Hq % Hkv) return false;
+  const long long group = Hq / Hkv;
+  const long long row_tiles = ceil_div(group * Lq, kBlockM);
+  const long long max_splits = ceil_div(Lk_max, kBlockN);
+  long long splits;
+  if (num_splits > 0) {
+    splits = num_splits < max_splits ? num_splits : max_splits;
+  } else {
+    // At least two waves of CTAs over the SMs, and chunks of at most 4096 keys
+    // so that ragged per-sequence lengths balance across the grid.
+    const long long units = (long long)B * Hkv * row_tiles;
+    long long want = ceil_div(2LL * num_sms(), units);
+    const long long by_len = ceil_div(Lk_max, 4096);
+    if (by_len > want) want = by_len;
+    splits = want < max_splits ? want : max_splits;
+  }
+  const long long chunk = ceil_div(ceil_div(Lk_max, splits), kBlockN) * kBlockN;
+  plan->chunk = (int)chunk;
+  plan->nsplit = (int)ceil_div(Lk_max, chunk);
+  plan->row_tiles = (int)row_tiles;
+  return true;
+}
+
+size_t ws_lse_offset(const SplitPlan& pl, long long nrows, int d) {
+  const size_t obytes = (size_t)pl.nsplit * (size_t)nrows * (size_t)d * 4;
+  return (obytes + 255) / 256 * 256;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* attn_status_string(attn_status_t s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+  }
+  return "ATTN_ERR_UNKNOWN";
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_kind,
+                       int window_l, int window_r, int draft_block, const int32_t* doc_ids,
+                       void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_DRAFT_BLOCK) return ATTN_ERR_INVALID_ARG;
+  if (window_l < -1 || window_r < -1) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_DRAFT_BLOCK && draft_block < 1) return ATTN_ERR_INVALID_ARG;
+  if (doc_ids && (!aligned(doc_ids, 4) || Lq > Lk)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (ceil_div(Lk, kBlockN) > attn::kMaxKvTiles) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hq > kMaxGridY) return ATTN_ERR_UNSUPPORTED;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof p);
+  p.o = o;
+  p.lse = lse;
+  p.doc_ids = doc_ids;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.group = Hq / Hkv;
+  p.mask_kind = mask_kind;
+  p.window_l = window_l;
+  p.window_r = window_r;
+  p.draft_block = mask_kind == ATTN_MASK_DRAFT_BLOCK ? draft_block : 1;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.q_tiles = (int)ceil_div(Lq, kBlockM);
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t dq[3] = {(uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq};
+  const uint64_t dk[3] = {(uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv};
+  if (!encode_bf16(&tq, q, 3, dq) || !encode_bf16(&tk, k, 3, dk) || !encode_bf16(&tv, v, 3, dk))
+    return ATTN_ERR_CUDA;
+
+  dim3 grid((unsigned)p.q_tiles, (unsigned)(B * Hq), 1);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = d == 64 ? attn::launch_fwd<64, false>(tq, tk, tv, p, grid, st)
+                          : attn::launch_fwd<128, false>(tq, tk, tv, p, grid, st);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_decode_num_splits(int B, int Hq, int Hkv, int Lq, int Lk_max, int d, int num_splits,
+                           int* chunk_keys) {
+  SplitPlan pl;
+  if (!plan_splits(B, Hq, Hkv, Lq, Lk_max, d, num_splits, &pl)) return -1;
+  if (chunk_keys) *chunk_keys = pl.chunk;
+  return pl.nsplit;
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk_max, int d,
+                                  int num_splits) {
+  SplitPlan pl;
+  if (!plan_splits(B, Hq, Hkv, Lq, Lk_max, d, num_splits, &pl)) return 0;
+  const long long nrows = (long long)B * Hq * Lq;
+  return ws_lse_offset(pl, nrows, d) + (size_t)pl.nsplit * (size_t)nrows * 4;
+}
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                                  void* o, float* lse, const int32_t* kv_lens, int B, int Hq,
+                                  int Hkv, int Lq, int Lk_max, int d, float scale, int num_splits,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  if (!q || !k_cache || !v_cache || !o || !lse || !kv_lens) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(kv_lens, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  SplitPlan pl;
+  if (!plan_splits(B, Hq, Hkv, Lq, Lk_max, d, num_splits, &pl)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (pl.chunk / kBlockN > attn::kMaxKvTiles) return ATTN_ERR_UNSUPPORTED;
+  const long long nrows = (long long)B * Hq * Lq;
+  if (nrows > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hkv * pl.row_tiles > kMaxGridY) return ATTN_ERR_UNSUPPORTED;
+  const size_t need = attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk_max, d, num_splits);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < need) return ATTN_ERR_WORKSPACE;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof p);
+  p.o = o;
+  p.lse = lse;
+  p.ws_o = reinterpret_cast<float*>(workspace);
+  p.ws_lse = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) +
+                                      ws_lse_offset(pl, nrows, d));
+  p.kv_lens = kv_lens;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lk = Lk_max;
+  p.group = Hq / Hkv;
+  p.mask_kind = ATTN_MASK_NONE;
+  p.window_l = -1;
+  p.window_r = -1;
+  p.draft_block = 1;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.chunk = pl.chunk;
+  p.nsplit = pl.nsplit;
+  p.row_tiles = pl.row_tiles;
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t dq[2] = {(uint64_t)d, (uint64_t)nrows};
+  const uint64_t dk[3] = {(uint64_t)d, (uint64_t)Lk_max, (uint64_t)B * Hkv};
+  if (!encode_bf16(&tq, q, 2, dq) || !encode_bf16(&tk, k_cache, 3, dk) ||
+      !encode_bf16(&tv, v_cache, 3, dk))
+    return ATTN_ERR_CUDA;
+
+  dim3 grid((unsigned)pl.nsplit, (unsigned)(B * Hkv * pl.row_tiles), 1);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = d == 64 ? attn::launch_fwd<64, true>(tq, tk, tv, p, grid, st)
+                          : attn::launch_fwd<128, true>(tq, tk, tv, p, grid, st);
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
+  e = d == 64 ? attn::launch_combine<64>(p, st) : attn::launch_combine<128>(p, st);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_get_device_error(void* stream, int* raw_bits) {
+  if (raw_bits) *raw_bits = 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return ATTN_ERR_CUDA;
+  int* word = attn::device_error_word();
+  if (!word) return ATTN_ERR_CUDA;
+  int bits = 0;
+  if (cudaMemcpy(&bits, word, sizeof bits, cudaMemcpyDeviceToHost) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(word, &zero, sizeof zero, cudaMemcpyHostToDevice) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  if (raw_bits) *raw_bits = bits;
+  if (bits & (attn::kDevErrTimeoutProducer | attn::kDevErrTimeoutMma |
+              attn::kDevErrTimeoutSoftmax))
+    return ATTN_ERR_TIMEOUT;
+  if (bits & attn::kDevErrBadKvLen) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+}  // extern "C"

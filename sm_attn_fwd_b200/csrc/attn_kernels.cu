@@ -1,0 +1,722 @@
+// Fused tiled attention forward for sm_100a (B200): prefill and split-KV decode.
+//
+// Method ("FlashAttention 2 原理与 PyTorch 实战", sections 一, 3.1, 3.2): a CTA owns
+// one 128-row query tile, streams 128-key K/V tiles through shared memory,
+// computes S = Q K^T, applies the mask, keeps a running row max m and sum l
+// (online softmax), rescales the accumulator and adds P V, so the N x N score
+// matrix never reaches HBM.  The mask is the mask_mod predicate of
+// "FlexAttention 是什么，以及 DFlash2 之谜的完整侦破" (section 1: causal, sliding
+// window, non-causal, document ids; section 3: the symmetric window and the
+// block-diffusion draft mask).  The split-KV decode (same page, section 1,
+// FlexDecoding / FlashDecoding) gives each CTA one chunk of the KV cache and
+// leaves a normalised partial output plus its log-sum-exp for the combine
+// kernel at the end of this file.
+//
+// B200 mapping (one CTA per SM, 192 threads):
+//   warp 0      TMA producer: Q once, then K and V tiles into a ring of stages
+//               (128-byte swizzled boxes, mbarrier transaction counts).
+//   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma:
+//               S_j = Q K_j^T (both operands in shared memory, fp32 in TMEM),
+//               O  += P_j V_j (P from TMEM, V from shared memory, MN-major).
+//   warps 2..5  softmax: thread r owns query row r (its TMEM lane), loads S_j,
+//               masks partial tiles, updates m and l in base 2, rescales O only
+//               when the running max grew by more than 2^8, writes P_j as bf16
+//               over S_j in TMEM, and finally stores O / l and the LSE.
+// Tensor memory: S double buffer at columns [0,128) and [128,256), O at
+// [256, 256 + d).  Key tiles that the mask empties entirely are never loaded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "attn_params.h"
+#include "ptx.cuh"
+
+namespace attn {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr uint32_t kTmemO = 256;
+// S (and P over it) double buffer: columns [0,128) and [128,256).
+__device__ __forceinline__ uint32_t tmem_s(int j) { return (j & 1) ? 128u : 0u; }
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when max grows by > 2^8
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D>
+struct Cfg {
+  static constexpr int kAtoms = D / 64;               // 128-byte swizzle atoms along d
+  static constexpr int kAtomBytes = kBlockN * 128;    // one atom column of a 128-row tile
+  static constexpr int kTileBytes = kBlockN * D * 2;  // one K or V tile (== Q tile)
+  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
+  // o_done, o_final, mma_drain
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 3;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kOffBits = kOffMisc + 64;
+  static constexpr int kBitWords = kMaxKvTiles / 32;
+  static constexpr int kSmemBytes = kOffBits + 2 * kBitWords * 4;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;  // slack for 1024-byte alignment
+};
+
+struct Misc {
+  uint32_t tmem_base;
+  int abort;
+  int n_tiles;
+  int t_lo;
+  int t_hi;
+};
+
+__device__ __forceinline__ long long floor_div_ll(long long a, long long b) {
+  return a >= 0 ? a / b : -((-a + b - 1) / b);
+}
+
+// Inclusive key range [lo, hi] the mask allows for a query at absolute
+// position pos, before the document test.  hi < lo means none.
+__device__ __forceinline__ void key_bounds(const FwdParams& p, long long pos, long long& lo,
+                                           long long& hi) {
+  lo = 0;
+  hi = (long long)p.Lk - 1;
+  if (p.mask_kind == kMaskCausal) {
+    hi = min(hi, pos);
+  } else if (p.mask_kind == kMaskDraftBlock) {
+    long long bd = p.draft_block;
+    hi = min(hi, (floor_div_ll(pos, bd) + 1) * bd - 1);
+  }
+  if (p.window_l >= 0) lo = max(lo, pos - (long long)p.window_l);
+  if (p.window_r >= 0) hi = min(hi, pos + (long long)p.window_r);
+}
+
+__device__ __forceinline__ bool bit_get(const uint32_t* bits, int i) {
+  return (bits[i >> 5] >> (i & 31)) & 1u;
+}
+
+template <int D>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int kk) {
+  // K-major operand, 16 elements of d per MMA: atom kk/4, 32 bytes per step inside it.
+  uint32_t addr = tile_saddr + (kk >> 2) * Cfg<D>::kAtomBytes + (kk & 3) * 32;
+  return ptx::smem_desc_sw128(addr, 16, 1024);
+}
+
+template <int D>
+__device__ __forceinline__ uint64_t desc_v_mnmajor(uint32_t tile_saddr, int kk) {
+  // V as the MN-major B operand of P V: 16 keys (two 8-row groups) per MMA step,
+  // 64-element d atoms 16 KB apart (leading offset), 8-key groups 1 KB apart (stride).
+  uint32_t addr = tile_saddr + kk * 2048;
+  return ptx::smem_desc_sw128(addr, Cfg<D>::kAtomBytes, 1024);
+}
+
+}  // namespace
+
+template <int D, bool kDecode>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + C::kStages;
+  uint64_t* v_full = k_empty + C::kStages;
+  uint64_t* v_empty = v_full + C::kStages;
+  uint64_t* s_full = v_empty + C::kStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_done = p_full + 2;
+  uint64_t* o_final = o_done + 1;
+  uint64_t* mma_drain = o_final + 1;
+  Misc* misc = reinterpret_cast<Misc*>(smem + C::kOffMisc);
+  uint32_t* empty_bits = reinterpret_cast<uint32_t*>(smem + C::kOffBits);
+  uint32_t* full_bits = empty_bits + C::kBitWords;
+  volatile int* abort_flag = &misc->abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ------------------------------------------------------------ work unit
+  int b, hkv, rows_valid, kv_z, q_coord_y, q_coord_z;
+  long long pos0 = 0;      // absolute position of tile row 0 (prefill)
+  int key_end;             // keys at or past this index are never visible
+  int t_lo, t_hi;          // candidate key tiles (absolute tile indices)
+  long long row_out0;      // flat output row of tile row 0
+  int split = 0;
+  if constexpr (kDecode) {
+    split = blockIdx.x;
+    const int bh = blockIdx.y / p.row_tiles;
+    const int rt = blockIdx.y % p.row_tiles;
+    b = bh / p.Hkv;
+    hkv = bh % p.Hkv;
+    int kv_len = p.kv_lens[b];
+    if (kv_len < 0 || kv_len > p.Lk) {
+      if (threadIdx.x == 0 && blockIdx.x == 0 && rt == 0) atomicOr(&g_device_error, kDevErrBadKvLen);
+      kv_len = kv_len < 0 ? 0 : p.Lk;
+    }
+    const int c0 = split * p.chunk;
+    if (c0 >= kv_len) return;  // this split holds no keys of sequence b (uniform exit)
+    key_end = min(c0 + p.chunk, kv_len);
+    rows_valid = min(kBlockM, p.group * p.Lq - rt * kBlockM);
+    row_out0 = ((long long)b * p.Hq + (long long)hkv * p.group) * p.Lq + (long long)rt * kBlockM;
+    q_coord_y = (int)row_out0;
+    q_coord_z = 0;
+    kv_z = b * p.Hkv + hkv;
+    t_lo = c0 / kBlockN;
+    t_hi = (key_end - 1) / kBlockN;
+  } else {
+    const int qt = p.q_tiles - 1 - (int)blockIdx.x;  // heaviest causal tiles first
+    const int bhq = blockIdx.y;
+    b = bhq / p.Hq;
+    const int hq = bhq % p.Hq;
+    hkv = hq / p.group;
+    const int q0 = qt * kBlockM;
+    rows_valid = min(kBlockM, p.Lq - q0);
+    row_out0 = (long long)bhq * p.Lq + q0;
+    q_coord_y = q0;
+    q_coord_z = bhq;
+    kv_z = b * p.Hkv + hkv;
+    key_end = p.Lk;
+    pos0 = (long long)p.Lk - p.Lq + q0;
+    long long lo_a, hi_a, lo_b, hi_b;
+    key_bounds(p, pos0, lo_a, hi_a);
+    key_bounds(p, pos0 + rows_valid - 1, lo_b, hi_b);
+    if (hi_b < lo_a || hi_b < 0) {
+      t_lo = 0;
+      t_hi = -1;
+    } else {
+      t_lo = (int)(lo_a / kBlockN);
+      t_hi = (int)(hi_b / kBlockN);
+    }
+  }
+
+  // ------------------------------------------------------------- prologue
+  if (warp == 0) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tm_q);
+      ptx::prefetch_tmap(&tm_k);
+      ptx::prefetch_tmap(&tm_v);
+      ptx::mbar_init(q_full, 1);
+      for (int s = 0; s < C::kStages; ++s) {
+        ptx::mbar_init(&k_full[s], 1);
+        ptx::mbar_init(&k_empty[s], 1);
+        ptx::mbar_init(&v_full[s], 1);
+        ptx::mbar_init(&v_empty[s], 1);
+      }
+      for (int s = 0; s < 2; ++s) {
+        ptx::mbar_init(&s_full[s], 1);
+        ptx::mbar_init(&p_full[s], 4 * 32);
+      }
+      ptx::mbar_init(o_done, 1);
+      ptx::mbar_init(o_final, 1);
+      ptx::mbar_init(mma_drain, 1);
+      misc->abort = 0;
+      misc->t_lo = t_lo;
+      misc->t_hi = t_hi;
+      ptx::fence_mbar_init();
+    }
+    // Tile classification: EMPTY tiles are skipped, FULL tiles need no mask.
+    const int ntc = t_hi - t_lo + 1;
+    int n_tiles = 0;
+    int qdmin = 0, qdmax = 0;
+    const int32_t* doc_b = nullptr;
+    if (!kDecode && p.doc_ids != nullptr && ntc > 0) {
+      doc_b = p.doc_ids + (long long)b * p.Lk;
+      int mn = 0x7fffffff, mx = (int)0x80000000;
+      for (int r = lane; r < rows_valid; r += 32) {
+        const int d = __ldg(doc_b + (pos0 + r));
+        mn = min(mn, d);
+        mx = max(mx, d);
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      qdmin = mn;
+      qdmax = mx;
+    }
+    long long lo_b = 0, hi_a = -1;
+    if (!kDecode) {
+      long long lo_a, hi_b;
+      key_bounds(p, pos0, lo_a, hi_a);
+      key_bounds(p, pos0 + rows_valid - 1, lo_b, hi_b);
+    }
+    for (int base = 0; base < ntc; base += 32) {
+      const int i = base + lane;
+      const int t = t_lo + i;
+      bool empty = false, full = false;
+      if (i < ntc) {
+        const long long k0 = (long long)t * kBlockN;
+        if constexpr (kDecode) {
+          full = (k0 + kBlockN <= key_end);
+        } else {
+          full = (k0 + kBlockN <= p.Lk) && (lo_b <= k0) && (hi_a >= k0 + kBlockN - 1);
+        }
+      }
+      if (doc_b != nullptr) {
+        // document ids: per tile min/max over the tile's keys (whole warp per tile)
+        for (int w = 0; w < 32 && base + w < ntc; ++w) {
+          const long long k0 = (long long)(t_lo + base + w) * kBlockN;
+          const int kend = (int)min(k0 + kBlockN, (long long)p.Lk);
+          int mn = 0x7fffffff, mx = (int)0x80000000;
+          for (long long kk = k0 + lane; kk < kend; kk += 32) {
+            const int d = __ldg(doc_b + kk);
+            mn = min(mn, d);
+            mx = max(mx, d);
+          }
+          for (int o = 16; o > 0; o >>= 1) {
+            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          }
+          if (lane == w) {
+            if (mx < qdmin || mn > qdmax) empty = true;
+            if (!(mn == mx && qdmin == qdmax && mn == qdmin)) full = false;
+          }
+        }
+      }
+      if (i >= ntc) empty = true;
+      const uint32_t eb = __ballot_sync(0xffffffffu, empty);
+      const uint32_t fb = __ballot_sync(0xffffffffu, full && !empty);
+      if (lane == 0) {
+        empty_bits[base >> 5] = eb;
+        full_bits[base >> 5] = fb;
+      }
+      n_tiles += __popc(~eb);
+    }
+    if (lane == 0) misc->n_tiles = n_tiles;
+  } else if (warp == 1) {
+    ptx::tmem_alloc(&misc->tmem_base, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+  const int n_tiles = misc->n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t kTx = C::kTileBytes;
+      ptx::mbar_arrive_expect_tx(q_full, kTx);
+      for (int a = 0; a < C::kAtoms; ++a) {
+        if constexpr (kDecode)
+          ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y);
+        else
+          ptx::tma_load_3d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y, q_coord_z);
+      }
+      int j = 0;
+      bool ok = true;
+      for (int t = t_lo; t <= t_hi && ok; ++t) {
+        if (bit_get(empty_bits, t - t_lo)) continue;
+        const int s = j % C::kStages;
+        const uint32_t ph = (uint32_t)(j / C::kStages) & 1u;
+        const int k0 = t * kBlockN;
+        ok = ptx::mbar_wait(&k_empty[s], ph ^ 1u, abort_flag, &g_device_error,
+                            kDevErrTimeoutProducer);
+        if (!ok) break;
+        ptx::mbar_arrive_expect_tx(&k_full[s], kTx);
+        for (int a = 0; a < C::kAtoms; ++a)
+          ptx::tma_load_3d(sK + s * C::kTileBytes + a * C::kAtomBytes, &tm_k, &k_full[s], a * 64,
+                           k0, kv_z);
+        ok = ptx::mbar_wait(&v_empty[s], ph ^ 1u, abort_flag, &g_device_error,
+                            kDevErrTimeoutProducer);
+        if (!ok) {
+          ++j;  // the K load of this tile is in flight; drain it below
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(&v_full[s], kTx);
+        for (int a = 0; a < C::kAtoms; ++a)
+          ptx::tma_load_3d(sV + s * C::kTileBytes + a * C::kAtomBytes, &tm_v, &v_full[s], a * 64,
+                           k0, kv_z);
+        ++j;
+      }
+      // Drain: every TMA write into shared memory must land before the CTA exits.
+      // In a normal run these phases have completed already.
+      int dummy_abort = 0;
+      ptx::mbar_wait(q_full, 0, &dummy_abort, nullptr, 0);
+      for (int jj = max(0, j - C::kStages); jj < j; ++jj) {
+        const int s = jj % C::kStages;
+        const uint32_t ph = (uint32_t)(jj / C::kStages) & 1u;
+        dummy_abort = 0;
+        ptx::mbar_wait(&k_full[s], ph, &dummy_abort, nullptr, 0);
+        dummy_abort = 0;
+        ptx::mbar_wait(&v_full[s], ph, &dummy_abort, nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+      constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(kBlockM, D, 0, 1);
+      const uint32_t q_saddr = ptx::smem_u32(sQ);
+      const uint32_t k_saddr = ptx::smem_u32(sK);
+      const uint32_t v_saddr = ptx::smem_u32(sV);
+      bool ok = ptx::mbar_wait(q_full, 0, abort_flag, &g_device_error, kDevErrTimeoutMma);
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % C::kStages;
+        const uint32_t ph = (uint32_t)(j / C::kStages) & 1u;
+        if (!ptx::mbar_wait(&k_full[s], ph, abort_flag, &g_device_error, kDevErrTimeoutMma))
+          return false;
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem + tmem_s(j);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          ptx::mma_ss(d_tmem, desc_kmajor<D>(q_saddr, kk),
+                      desc_kmajor<D>(k_saddr + s * C::kTileBytes, kk), kIdescS, kk > 0 ? 1u : 0u);
+        }
+        ptx::mma_commit(&s_full[j & 1]);
+        ptx::mma_commit(&k_empty[s]);
+        return true;
+      };
+      if (ok) ptx::tc_fence_after();
+      if (ok) ok = issue_s(0);
+      for (int j = 0; j < n_tiles && ok; ++j) {
+        if (j + 1 < n_tiles) {
+          ok = issue_s(j + 1);
+          if (!ok) break;
+        }
+        const int s = j % C::kStages;
+        ok = ptx::mbar_wait(&p_full[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, &g_device_error,
+                            kDevErrTimeoutMma);
+        if (!ok) break;
+        ok = ptx::mbar_wait(&v_full[s], (uint32_t)(j / C::kStages) & 1u, abort_flag,
+                            &g_device_error, kDevErrTimeoutMma);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const uint32_t p_tmem = tmem + tmem_s(j);
+#pragma unroll
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          // P occupies 64 columns: two bf16 per 32-bit column, 16 keys per 8 columns.
+          ptx::mma_ts(tmem + kTmemO, p_tmem + kk * 8,
+                      desc_v_mnmajor<D>(v_saddr + s * C::kTileBytes, kk), kIdescPV,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::mma_commit(o_done);
+        ptx::mma_commit(&v_empty[s]);
+      }
+      ptx::mma_commit(o_final);
+      // Wait for every MMA to finish before tensor memory is released.
+      ptx::mma_commit(mma_drain);
+      int dummy_abort = 0;
+      ptx::mbar_wait(mma_drain, 0, &dummy_abort, nullptr, 0);
+    }
+  } else {
+    // ----------------------------------------------------------- softmax
+    const int quarter = warp & 3;           // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;      // tile row == TMEM lane
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
+    const bool row_ok = r < rows_valid;
+    const float c = p.scale_log2;
+
+    // visible key range of this row, before the document test
+    long long row_lo = 0, row_hi = -1;
+    int row_doc = 0;
+    const int32_t* doc_b = nullptr;
+    if (row_ok) {
+      if constexpr (kDecode) {
+        row_lo = 0;
+        row_hi = key_end - 1;
+      } else {
+        const long long pos = pos0 + r;
+        key_bounds(p, pos, row_lo, row_hi);
+        if (p.doc_ids != nullptr) {
+          doc_b = p.doc_ids + (long long)b * p.Lk;
+          row_doc = __ldg(doc_b + pos);
+        }
+      }
+    }
+
+    float m_ref = -INFINITY;  // reference max (base-2 scaled units)
+    float l = 0.0f;
+    int j = 0;
+    bool ok = true;
+    for (int t = t_lo; t <= t_hi && ok; ++t) {
+      if (bit_get(empty_bits, t - t_lo)) continue;
+      const bool full = bit_get(full_bits, t - t_lo);
+      const long long k0 = (long long)t * kBlockN;
+      ok = ptx::mbar_wait(&s_full[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag, &g_device_error,
+                          kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);  // warp-collective TMEM access below
+      if (!ok) break;
+      ptx::tc_fence_after();
+
+      float s[kBlockN];
+      {
+        uint32_t raw[32];
+#pragma unroll
+        for (int cc = 0; cc < kBlockN / 32; ++cc) {
+          ptx::tmem_ld32(t_row + tmem_s(j) + cc * 32, raw);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(raw[i]);
+        }
+      }
+      if (!full) {
+#pragma unroll
+        for (int i = 0; i < kBlockN; ++i) {
+          const long long key = k0 + i;
+          bool vis = (key >= row_lo) && (key <= row_hi);
+          if (doc_b != nullptr && vis) vis = (__ldg(doc_b + key) == row_doc);
+          s[i] = vis ? s[i] : -INFINITY;
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < kBlockN; ++i) mx = fmaxf(mx, s[i]);
+      const float m_tile = mx * c;
+      const float m_new = fmaxf(m_ref, m_tile);
+      const bool need = m_new > m_ref + kRescaleThreshold;
+      const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;  // 0 when m_ref = -inf
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O holds P_{<j} V; it must be final before it is rescaled.
+        ok = ptx::mbar_wait(o_done, (uint32_t)(j - 1) & 1u, abort_flag, &g_device_error,
+                            kDevErrTimeoutSoftmax);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t raw[32];
+          ptx::tmem_ld32(t_row + kTmemO + cc * 32, raw);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+          ptx::tmem_st32(t_row + kTmemO + cc * 32, raw);
+        }
+      }
+      if (need) {
+        l *= alpha;
+        m_ref = m_new;
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+      float rowsum = 0.0f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t packed[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float p0 = ptx::ex2(fmaf(s[h * 64 + 2 * i], c, -m_use));
+          const float p1 = ptx::ex2(fmaf(s[h * 64 + 2 * i + 1], c, -m_use));
+          rowsum += p0 + p1;
+          packed[i] = ptx::pack_bf16x2(p0, p1);
+        }
+        ptx::tmem_st32(t_row + tmem_s(j) + h * 32, packed);
+      }
+      l += rowsum;
+      if constexpr (kDecode) {
+        // Keys past the end of this sequence: their V rows may hold anything
+        // (even NaN), and 0 * NaN would poison O.  Zero them in shared memory.
+        if (!full) {
+          const int s_stage = j % C::kStages;
+          const bool zero_row = (k0 + r >= key_end);
+          if (__any_sync(0xffffffffu, zero_row)) {
+            ok = ptx::mbar_wait(&v_full[s_stage], (uint32_t)(j / C::kStages) & 1u, abort_flag,
+                                &g_device_error, kDevErrTimeoutSoftmax);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            if (zero_row) {
+#pragma unroll
+              for (int a = 0; a < C::kAtoms; ++a) {
+                uint4* row_ptr = reinterpret_cast<uint4*>(sV + s_stage * C::kTileBytes +
+                                                          a * C::kAtomBytes + r * 128);
+#pragma unroll
+                for (int q = 0; q < 8; ++q) row_ptr[q] = make_uint4(0, 0, 0, 0);
+              }
+              ptx::fence_proxy_async_smem();
+            }
+          }
+        }
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&p_full[j & 1]);
+      ++j;
+    }
+
+    // ---------------------------------------------------------- epilogue
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok && n_tiles > 0) {
+      ok = ptx::mbar_wait(o_final, 0, abort_flag, &g_device_error, kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+      ptx::tc_fence_after();
+    }
+    const bool have = ok && n_tiles > 0 && l > 0.0f;
+    const float inv_l = have ? 1.0f / l : 0.0f;
+    const float lse_row = have ? (m_ref + ptx::lg2(l)) * kLn2 : -INFINITY;
+    const long long out_row = row_out0 + r;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t raw[32];
+      if (ok && n_tiles > 0) {
+        ptx::tmem_ld32(t_row + kTmemO + cc * 32, raw);
+        ptx::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) raw[i] = 0u;
+      }
+      if (row_ok) {
+        if constexpr (kDecode) {
+          float* dst = p.ws_o + ((long long)split * p.B * p.Hq * p.Lq + out_row) * D + cc * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            float4 v4 = make_float4(__uint_as_float(raw[i]) * inv_l,
+                                    __uint_as_float(raw[i + 1]) * inv_l,
+                                    __uint_as_float(raw[i + 2]) * inv_l,
+                                    __uint_as_float(raw[i + 3]) * inv_l);
+            *reinterpret_cast<float4*>(dst + i) = v4;
+          }
+        } else {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + out_row * D + cc * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v4;
+            v4.x = ptx::pack_bf16x2(__uint_as_float(raw[i]) * inv_l,
+                                    __uint_as_float(raw[i + 1]) * inv_l);
+            v4.y = ptx::pack_bf16x2(__uint_as_float(raw[i + 2]) * inv_l,
+                                    __uint_as_float(raw[i + 3]) * inv_l);
+            v4.z = ptx::pack_bf16x2(__uint_as_float(raw[i + 4]) * inv_l,
+                                    __uint_as_float(raw[i + 5]) * inv_l);
+            v4.w = ptx::pack_bf16x2(__uint_as_float(raw[i + 6]) * inv_l,
+                                    __uint_as_float(raw[i + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + i) = v4;
+          }
+        }
+      }
+    }
+    if (row_ok) {
+      if constexpr (kDecode)
+        p.ws_lse[(long long)split * p.B * p.Hq * p.Lq + out_row] = lse_row;
+      else
+        p.lse[out_row] = lse_row;
+    }
+  }
+
+  // ------------------------------------------------------------- teardown
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Split-KV combine (the LSE-weighted merge of FlashDecoding-style partials):
+//   LSE = log sum_s exp(LSE_s),  O = sum_s exp(LSE_s - LSE) O_s.
+// One warp per output row; lane i owns d/32 consecutive elements.
+template <int D>
+__global__ void __launch_bounds__(256) attn_decode_combine_kernel(const FwdParams p) {
+  constexpr int kPer = D / 32;
+  constexpr float kLog2e = 1.44269504088896340736f;
+  const long long nrows = (long long)p.B * p.Hq * p.Lq;
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= nrows) return;
+  const int b = (int)(row / ((long long)p.Hq * p.Lq));
+  int kv_len = p.kv_lens[b];
+  kv_len = kv_len < 0 ? 0 : (kv_len > p.Lk ? p.Lk : kv_len);
+  const int ns = (kv_len + p.chunk - 1) / p.chunk;
+  float mx = -INFINITY;
+  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, p.ws_lse[(long long)s * nrows + row]);
+  float acc[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+  float sum = 0.0f;
+  if (mx != -INFINITY) {
+    for (int s = 0; s < ns; ++s) {
+      const float ls = p.ws_lse[(long long)s * nrows + row];
+      if (ls == -INFINITY) continue;
+      const float w = ptx::ex2((ls - mx) * kLog2e);
+      sum += w;
+      const float* src = p.ws_o + ((long long)s * nrows + row) * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+        acc[2] += w * v.z;
+        acc[3] += w * v.w;
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+      }
+    }
+  }
+  const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
+  __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    uint2 v;
+    v.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    v.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = v;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lane == 0) p.lse[row] = sum > 0.0f ? mx + ptx::lg2(sum) * kLn2 : -INFINITY;
+}
+
+// ------------------------------------------------------------- launchers
+template <int D, bool kDecode>
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, dim3 grid, cudaStream_t stream) {
+  auto kern = attn_fwd_kernel<D, kDecode>;
+  constexpr int smem = Cfg<D>::kSmemAlloc;
+  // The shared-memory opt-in is set once per device, outside any stream capture
+  // that a later call may be part of.
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream) {
+  const long long nrows = (long long)p.B * p.Hq * p.Lq;
+  const int warps = 8;
+  const long long blocks = (nrows + warps - 1) / warps;
+  attn_decode_combine_kernel<D><<<(unsigned)blocks, warps * 32, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_fwd<64, false>(const CUtensorMap&, const CUtensorMap&,
+                                           const CUtensorMap&, const FwdParams&, dim3,
+                                           cudaStream_t);
+template cudaError_t launch_fwd<128, false>(const CUtensorMap&, const CUtensorMap&,
+                                            const CUtensorMap&, const FwdParams&, dim3,
+                                            cudaStream_t);
+template cudaError_t launch_fwd<64, true>(const CUtensorMap&, const CUtensorMap&,
+                                          const CUtensorMap&, const FwdParams&, dim3,
+                                          cudaStream_t);
+template cudaError_t launch_fwd<128, true>(const CUtensorMap&, const CUtensorMap&,
+                                           const CUtensorMap&, const FwdParams&, dim3,
+                                           cudaStream_t);
+template cudaError_t launch_combine<64>(const FwdParams&, cudaStream_t);
+template cudaError_t launch_combine<128>(const FwdParams&, cudaStream_t);
+
+int* device_error_word() {
+  int* ptr = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr), g_device_error) != cudaSuccess)
+    return nullptr;
+  return ptr;
+}
+
+}  // namespace attn

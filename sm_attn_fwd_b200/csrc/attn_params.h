@@ -1,0 +1,45 @@
+// Launch parameters shared by the host planner (attn_api.cu) and the kernels
+// (attn_kernels.cu).  Plain data only.
+#pragma once
+
+#include <cstdint>
+
+namespace attn {
+
+constexpr int kBlockM = 128;     // query rows per tile (tcgen05 M)
+constexpr int kBlockN = 128;     // keys per tile (N of S = QK^T, K of O += PV)
+constexpr int kMaxKvTiles = 4096;  // key tiles one work unit may span (Lk <= 512K)
+
+enum MaskKind : int { kMaskNone = 0, kMaskCausal = 1, kMaskDraftBlock = 2 };
+
+// Error bits the kernels OR into the device error word.
+enum DeviceError : int {
+  kDevErrTimeoutProducer = 1 << 0,
+  kDevErrTimeoutMma = 1 << 1,
+  kDevErrTimeoutSoftmax = 1 << 2,
+  kDevErrBadKvLen = 1 << 3,
+};
+
+struct FwdParams {
+  // outputs
+  void* o;          // prefill: bf16 [B, Hq, Lq, d]; decode: unused
+  float* lse;       // prefill: fp32 [B, Hq, Lq]; decode: unused
+  float* ws_o;      // decode: fp32 [nsplit, B*Hq*Lq, d] normalised partial outputs
+  float* ws_lse;    // decode: fp32 [nsplit, B*Hq*Lq] partial log-sum-exp
+  // optional inputs
+  const int32_t* doc_ids;  // [B, Lk] or null
+  const int32_t* kv_lens;  // decode: [B]
+  // shapes
+  int B, Hq, Hkv, Lq, Lk;  // decode: Lk = Lk_max
+  int group;               // Hq / Hkv
+  // mask (prefill)
+  int mask_kind, window_l, window_r, draft_block;
+  float scale_log2;  // softmax scale * log2(e)
+  // decode split plan
+  int chunk;         // keys per split (multiple of kBlockN)
+  int nsplit;        // splits covering Lk_max
+  int row_tiles;     // 128-row tiles per (b, kv head): ceil(group * Lq / 128)
+  int q_tiles;       // prefill: ceil(Lq / 128)
+};
+
+}  // namespace attn

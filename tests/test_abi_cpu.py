@@ -1,0 +1,114 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/attn.h declares, and rejects invalid arguments on the host before
+touching CUDA (so these calls are safe on a machine with no device)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import sm_attn_fwd_b200 as ab
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_documented_entry_points():
+    assert set(declared_functions()) == set(ab.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ab.load_library()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", ab.lib_path()], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (attn_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_status_strings():
+    names = {ab.ATTN_OK: "ATTN_OK", ab.ATTN_ERR_INVALID_ARG: "ATTN_ERR_INVALID_ARG",
+             ab.ATTN_ERR_UNSUPPORTED: "ATTN_ERR_UNSUPPORTED",
+             ab.ATTN_ERR_WORKSPACE: "ATTN_ERR_WORKSPACE", ab.ATTN_ERR_CUDA: "ATTN_ERR_CUDA",
+             ab.ATTN_ERR_TIMEOUT: "ATTN_ERR_TIMEOUT"}
+    for code, name in names.items():
+        assert ab.attn_status_string(code) == name
+    assert ab.attn_status_string(99) == "ATTN_ERR_UNKNOWN"
+
+
+# Fake, 256-byte aligned addresses: validation must reject the call before
+# any pointer is dereferenced or any CUDA call is made.
+A = ctypes.c_void_p(0x10000)
+M = ctypes.c_void_p(0x10008)  # misaligned for 16-byte operands
+
+
+def _fwd(**kw):
+    args = dict(q=A, k=A, v=A, o=A, lse=A, B=1, Hq=2, Hkv=1, Lq=8, Lk=8, d=64, scale=0.125,
+                mask=0, wl=-1, wr=-1, bd=1, doc=None, stream=None)
+    args.update(kw)
+    return ab.load_library().attn_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"],
+                                      args["B"], args["Hq"], args["Hkv"], args["Lq"], args["Lk"],
+                                      args["d"], args["scale"], args["mask"], args["wl"],
+                                      args["wr"], args["bd"], args["doc"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), ab.ATTN_ERR_INVALID_ARG),
+    (dict(o=M), ab.ATTN_ERR_INVALID_ARG),
+    (dict(B=0), ab.ATTN_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), ab.ATTN_ERR_INVALID_ARG),
+    (dict(Lq=0), ab.ATTN_ERR_INVALID_ARG),
+    (dict(scale=0.0), ab.ATTN_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), ab.ATTN_ERR_INVALID_ARG),
+    (dict(mask=3), ab.ATTN_ERR_INVALID_ARG),
+    (dict(wl=-2), ab.ATTN_ERR_INVALID_ARG),
+    (dict(mask=2, bd=0), ab.ATTN_ERR_INVALID_ARG),
+    (dict(doc=A, Lq=9, Lk=8), ab.ATTN_ERR_INVALID_ARG),
+    (dict(d=96), ab.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), ab.ATTN_ERR_UNSUPPORTED),
+    (dict(Lk=4096 * 128 + 1), ab.ATTN_ERR_UNSUPPORTED),
+])
+def test_attn_fwd_rejects_on_host(kw, status):
+    assert _fwd(**kw) == status
+
+
+def test_decode_split_plan_and_workspace_arithmetic():
+    lib = ab.load_library()
+    chunk = ctypes.c_int(0)
+    # explicit split count: chunk = 128 * ceil(ceil(Lk / s) / 128)
+    n = lib.attn_decode_num_splits(2, 16, 2, 1, 1000, 128, 3, ctypes.byref(chunk))
+    assert (n, chunk.value) == (3, 384)
+    n = lib.attn_decode_num_splits(2, 16, 2, 1, 1000, 128, 100, ctypes.byref(chunk))
+    assert (n, chunk.value) == (8, 128)           # capped at ceil(1000 / 128)
+    # library choice: chunks never exceed 4096 keys and cover Lk_max
+    n = lib.attn_decode_num_splits(64, 64, 8, 1, 32768, 128, 0, ctypes.byref(chunk))
+    assert chunk.value <= 4096 and chunk.value % 128 == 0 and n * chunk.value >= 32768
+    ws = lib.attn_decode_workspace_size(2, 16, 2, 1, 1000, 128, 3)
+    nrows = 2 * 16 * 1
+    o_bytes = 3 * nrows * 128 * 4
+    assert ws == (o_bytes + 255) // 256 * 256 + 3 * nrows * 4
+    assert lib.attn_decode_num_splits(2, 16, 3, 1, 1000, 128, 0, None) == -1
+    assert lib.attn_decode_workspace_size(0, 16, 2, 1, 1000, 128, 0) == 0
+
+
+def test_decode_rejects_on_host():
+    lib = ab.load_library()
+    args = [A, A, A, A, A, A, 2, 16, 2, 1, 1000, 128, 0.125, 0, A, 1 << 30, None]
+    assert lib.attn_decode_splitkv(*args[:5], None, *args[6:]) == ab.ATTN_ERR_INVALID_ARG
+    bad_d = list(args)
+    bad_d[11] = 80
+    assert lib.attn_decode_splitkv(*bad_d) == ab.ATTN_ERR_UNSUPPORTED
+    small_ws = list(args)
+    small_ws[15] = 64
+    assert lib.attn_decode_splitkv(*small_ws) == ab.ATTN_ERR_WORKSPACE
+    no_ws = list(args)
+    no_ws[14] = None
+    assert lib.attn_decode_splitkv(*no_ws) == ab.ATTN_ERR_WORKSPACE

@@ -1,0 +1,177 @@
+"""GPU parity of attn_fwd (prefill) against the oracle, through the C ABI."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sm_attn_fwd_b200 as ab
+from tests.gpu_helpers import compare, sample_rows, to_dev
+from workloads import (CAUSAL_4K, CAUSAL_32K_GQA, DRAFT_WINDOW_DOC, DRAFT_WINDOW_DOC_FULL, TINY,
+                       make_inputs, random_case)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(q, k, v, **kw):
+    qd, kd, vd = to_dev(q, k, v)
+    doc = kw.pop("doc_ids", None)
+    docd = None if doc is None else doc.cuda().contiguous()
+    o, lse = ab.attn_fwd(qd, kd, vd, doc_ids=docd, **kw)
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    return o, lse
+
+
+def test_tiny_config_full():
+    """B=1, H=2, L=128, d=64, no mask, scale 1/8: every element."""
+    inp = make_inputs(TINY)
+    o, lse = _run(inp.q, inp.k, inp.v, scale=TINY.softmax_scale)
+    ro, rl = oracle.attn_fwd(inp.q, inp.k, inp.v, scale=TINY.softmax_scale)
+    compare(o, lse, ro, rl, "tiny")
+
+
+RAGGED = [
+    # seed, B, Hq, Hkv, Lq, Lk, d, mask, window, bd, doc
+    (1, 1, 2, 2, 1, 1, 64, "none", (-1, -1), 1, False),
+    (2, 2, 3, 1, 200, 333, 64, "none", (-1, -1), 1, False),
+    (3, 1, 4, 2, 300, 300, 128, "causal", (-1, -1), 1, False),
+    (4, 2, 2, 2, 129, 257, 64, "causal", (-1, -1), 1, False),
+    (5, 1, 2, 1, 385, 385, 128, "causal", (100, 0), 1, False),
+    (6, 1, 2, 2, 260, 260, 64, "none", (37, 37), 1, False),
+    (7, 2, 2, 2, 300, 300, 128, "draft", (-1, -1), 16, False),
+    (8, 1, 4, 4, 16, 2064, 128, "draft", (512, 512), 16, True),
+    (9, 2, 2, 2, 500, 500, 64, "causal", (-1, -1), 1, True),
+    (10, 1, 2, 2, 600, 200, 64, "causal", (-1, -1), 1, False),   # Lq > Lk: empty rows
+    (11, 1, 2, 2, 130, 1000, 128, "draft", (3, 200), 7, False),
+    (12, 1, 8, 2, 256, 1024, 64, "causal", (-1, -1), 1, False),
+]
+
+
+@pytest.mark.parametrize("case", RAGGED, ids=lambda c: f"s{c[0]}_{c[7]}_lq{c[4]}_lk{c[5]}_d{c[6]}")
+def test_ragged_shapes_and_masks(case):
+    seed, B, Hq, Hkv, Lq, Lk, d, mask, window, bd, doc = case
+    q, k, v, doc_ids, _ = random_case(seed, B, Hq, Hkv, Lq, Lk, d, doc_split=doc, n_docs=3)
+    kw = dict(scale=1.0 / math.sqrt(d), mask=mask, window=window, draft_block=bd)
+    o, lse = _run(q, k, v, doc_ids=doc_ids, **kw)
+    ro, rl = oracle.attn_fwd(q, k, v, doc_ids=doc_ids, **kw)
+    compare(o, lse, ro, rl, str(case))
+
+
+@pytest.mark.parametrize("case", [
+    (64, 257, 300, "causal", (-1, -1), 1, False),
+    (128, 200, 700, "draft", (40, 40), 16, True),
+    (64, 520, 520, "none", (130, 5), 1, True),
+    (128, 16, 2064, "draft", (512, 512), 16, True),
+])
+def test_mask_recovered_bit_exactly(case):
+    """Q = 0 makes every visible key equally likely; V = one-hot columns then
+    reads the mask back: O[i, c] != 0 exactly when key t*d + c is visible for
+    chunk t.  LSE = ln(count) checks the per-row counts."""
+    d, Lq, Lk, mask, window, bd, doc = case
+    _, _, _, doc_ids, _ = random_case(5, 1, 1, 1, Lq, Lk, d, doc_split=doc, n_docs=4)
+    want = oracle.mask(1, Lq, Lk, mask=mask, window=window, draft_block=bd, doc_ids=doc_ids)[0]
+    q = torch.zeros(1, 1, Lq, d, dtype=torch.bfloat16)
+    k = torch.randn(1, 1, Lk, d, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    got = np.zeros((Lq, Lk), dtype=bool)
+    lse_all = None
+    for t in range((Lk + d - 1) // d):
+        v = torch.zeros(1, 1, Lk, d)
+        keys = np.arange(t * d, min((t + 1) * d, Lk))
+        v[0, 0, keys, keys - t * d] = 1.0
+        o, lse = _run(q, k * 0, v.to(torch.bfloat16), scale=0.125, mask=mask, window=window,
+                      draft_block=bd, doc_ids=doc_ids)
+        oc = o[0, 0].float().cpu().numpy()
+        got[:, keys] = oc[:, : len(keys)] != 0.0
+        lse_all = lse[0, 0].cpu().numpy()
+    assert np.array_equal(got, want)
+    cnt = want.sum(-1)
+    has = cnt > 0
+    assert np.all(np.isneginf(lse_all[~has]))
+    np.testing.assert_allclose(lse_all[has], np.log(cnt[has]), atol=1e-5)
+
+
+def test_output_guard_bytes_untouched():
+    """Stores stay inside O and LSE: sentinel bytes after both survive."""
+    B, H, L, d = 1, 2, 300, 64
+    q, k, v, _, _ = random_case(3, B, H, H, L, L, d)
+    qd, kd, vd = to_dev(q, k, v)
+    n_o, n_l = B * H * L * d, B * H * L
+    o_buf = torch.full((n_o + 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((n_l + 1024,), 7.0, dtype=torch.float32, device="cuda")
+    o = o_buf[:n_o].view(B, H, L, d)
+    lse = l_buf[:n_l].view(B, H, L)
+    ab.attn_fwd(qd, kd, vd, mask="causal", o=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.all(o_buf[n_o:] == 7.0) and torch.all(l_buf[n_l:] == 7.0)
+    ro, rl = oracle.attn_fwd(q, k, v, mask="causal")
+    compare(o, lse, ro, rl, "guard")
+
+
+def test_config_causal_4k_sampled():
+    cfg = CAUSAL_4K
+    inp = make_inputs(cfg)
+    o, lse = _run(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask)
+    rows = sample_rows(cfg.B, cfg.Hq, cfg.Lq, 24, seed=1)
+    ro, rl = oracle.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask,
+                             rows=rows)
+    compare(o.reshape(-1, cfg.d)[torch.from_numpy(rows).cuda()],
+            lse.reshape(-1)[torch.from_numpy(rows).cuda()], ro, rl, cfg.name)
+
+
+def test_config_causal_32k_gqa_sampled():
+    cfg = CAUSAL_32K_GQA
+    inp = make_inputs(cfg)
+    o, lse = _run(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask)
+    rows = sample_rows(cfg.B, cfg.Hq, cfg.Lq, 6, seed=2)
+    ro, rl = oracle.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask,
+                             rows=rows)
+    idx = torch.from_numpy(rows).cuda()
+    compare(o.reshape(-1, cfg.d)[idx], lse.reshape(-1)[idx], ro, rl, cfg.name)
+
+
+@pytest.mark.parametrize("cfg", [DRAFT_WINDOW_DOC, DRAFT_WINDOW_DOC_FULL], ids=lambda c: c.name)
+def test_config_draft_window_doc_full(cfg):
+    inp = make_inputs(cfg)
+    kw = dict(scale=cfg.softmax_scale, mask=cfg.mask, window=cfg.window,
+              draft_block=cfg.draft_block)
+    o, lse = _run(inp.q, inp.k, inp.v, doc_ids=inp.doc_ids, **kw)
+    ro, rl = oracle.attn_fwd(inp.q, inp.k, inp.v, doc_ids=inp.doc_ids, **kw)
+    compare(o, lse, ro, rl, cfg.name)
+
+
+def test_invalid_arguments_launch_nothing():
+    q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 3, 8, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ab.AttnError) as e:
+        ab.attn_fwd(q, k, k)                        # Hq % Hkv != 0
+    assert e.value.status == ab.ATTN_ERR_INVALID_ARG
+    q96 = torch.zeros(1, 2, 8, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(ab.AttnError) as e:
+        ab.attn_fwd(q96, q96, q96)                  # d = 96 not built
+    assert e.value.status == ab.ATTN_ERR_UNSUPPORTED
+    with pytest.raises(ab.AttnError) as e:
+        ab.attn_fwd(q, q, q, mask="draft", draft_block=0)
+    assert e.value.status == ab.ATTN_ERR_INVALID_ARG
+
+
+def test_capturable_in_cuda_graph():
+    """The call allocates nothing and never synchronises, so it can be captured."""
+    q, k, v, _, _ = random_case(9, 1, 2, 2, 256, 256, 64)
+    qd, kd, vd = to_dev(q, k, v)
+    o = torch.empty_like(qd)
+    lse = torch.empty(1, 2, 256, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ab.attn_fwd(qd, kd, vd, mask="causal", o=o, lse=lse, stream=s)  # warm-up (attributes)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        ab.attn_fwd(qd, kd, vd, mask="causal", o=o, lse=lse, stream=s)
+    o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    ro, rl = oracle.attn_fwd(q, k, v, mask="causal")
+    compare(o, lse, ro, rl, "graph")

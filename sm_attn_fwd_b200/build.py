@@ -36,6 +36,11 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
+def source_digest() -> str:
+    """Digest of the kernel sources and flags (identifies a profiled build)."""
+    return _digest()
+
+
 def _digest() -> str:
     h = hashlib.sha256()
     for name in SOURCES + HEADERS:

@@ -354,8 +354,8 @@ def main_reference(args, world, rank):
     vals = []
     info = None
     for i in range(args.warmup + args.steps):
-        info = cpu_oracle_sample(cfg, target_s=max(1.0, 60.0 / max(1, args.steps + args.warmup)),
-                                 inp=inp)
+        info = cpu_oracle_sample(
+            cfg, target_s=max(0.5, args.ref_seconds / max(1, args.steps + args.warmup)), inp=inp)
         if i >= args.warmup:
             vals.append(info["value"])
     v = statistics.median(vals)
@@ -382,6 +382,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None,
                     help="with --only: set the batch size B (smaller profiling case)")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="--impl reference: total CPU seconds across all steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" and args.only is None else args.warmup

@@ -148,6 +148,38 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
                                   void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_decode_splitkv_noalloc — attn_decode_splitkv for callers that cannot
+ * allocate device memory.  (No counterpart on the pages: this is a library
+ * convenience, not part of the method.)
+ *
+ * Some callers cannot call cudaMalloc or any other allocator: for example a
+ * plugin inside a serving process whose device memory is all handed out by
+ * the host application's own pool, or a latency-critical decode loop where an
+ * allocation (which may synchronise the device) is not allowed.  They still
+ * own and pass q, k_cache, v_cache, o, lse and kv_lens, with the meaning,
+ * layout and rules of attn_decode_splitkv; the split workspace comes from a
+ * fixed 32 MiB array in device memory that the library declares itself.
+ *   - Every GPU that loads the library holds that array until the process
+ *     exits.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make this first call before any stream capture.
+ *   - Requests whose attn_decode_workspace_size(...) exceeds 32 MiB return
+ *     ATTN_ERR_WORKSPACE and launch nothing (e.g. B=64, Hq=64, Lq=1,
+ *     Lk_max=32768, d=128 needs 16.9 MB and fits; the Lq=16 variant does not).
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Nothing in it needs to start at zero (every value the combine reads is
+ *     written first by the same call), but two calls that overlap on the GPU
+ *     (different streams, or different host threads) race on it: serialise
+ *     them.
+ * Errors: as attn_decode_splitkv, plus ATTN_ERR_WORKSPACE above.
+ */
+attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* k_cache,
+                                          const void* v_cache, void* o, float* lse,
+                                          const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
+                                          int Lk_max, int d, float scale, int num_splits,
+                                          void* stream);
+
+/*
  * attn_get_device_error — synchronise `stream`, then read and clear the
  * device error word of the current device.  Returns ATTN_OK, ATTN_ERR_TIMEOUT
  * (a kernel abandoned a bounded wait), ATTN_ERR_INVALID_ARG (a kv_lens entry

@@ -26,7 +26,8 @@ __all__ = [
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
     "attn_fwd", "attn_decode_splitkv", "attn_decode_num_splits",
-    "attn_decode_workspace_size", "attn_get_device_error", "attn_status_string",
+    "attn_decode_workspace_size", "attn_decode_splitkv_noalloc", "attn_get_device_error",
+    "attn_status_string",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -44,7 +45,8 @@ _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 
 EXPORTED_SYMBOLS = (
     "attn_fwd", "attn_decode_num_splits", "attn_decode_workspace_size",
-    "attn_decode_splitkv", "attn_get_device_error", "attn_status_string",
+    "attn_decode_splitkv", "attn_decode_splitkv_noalloc", "attn_get_device_error",
+    "attn_status_string",
 )
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -84,6 +86,9 @@ def load_library():
         lib.attn_decode_splitkv.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
                                             i32, P, sz, P]
         lib.attn_decode_splitkv.restype = i32
+        lib.attn_decode_splitkv_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                                    i32, f32, i32, P]
+        lib.attn_decode_splitkv_noalloc.restype = i32
         lib.attn_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         lib.attn_get_device_error.restype = i32
         lib.attn_status_string.argtypes = [i32]
@@ -190,6 +195,32 @@ def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, *, scale=None, num_splits=
         workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_decode_splitkv_noalloc(q, k_cache, v_cache, kv_lens, *, scale=None, num_splits=0,
+                                o=None, lse=None, stream=None):
+    """Split-KV decode with the library's fixed device workspace (see
+    ``attn_decode_splitkv_noalloc`` in include/attn.h): for callers that
+    cannot allocate.  ``o`` and ``lse`` should be passed in by such callers;
+    they are only allocated here as a convenience when omitted."""
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_bf16(name, t)
+    if kv_lens.dtype != torch.int32 or not kv_lens.is_cuda or not kv_lens.is_contiguous():
+        raise ValueError("kv_lens must be a contiguous int32 CUDA tensor [B]")
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk_max, _ = k_cache.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_decode_splitkv_noalloc(
+        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), _ptr(kv_lens), B, Hq, Hkv,
+        Lq, Lk_max, d, float(scale), int(num_splits), _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_decode_splitkv_noalloc")
     return o, lse
 
 

@@ -19,6 +19,9 @@ cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap
                        const FwdParams&, dim3, cudaStream_t);
 template <int D>
 cudaError_t launch_combine(const FwdParams&, cudaStream_t);
+template <int D>
+cudaError_t launch_prefill(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                           const FwdParams&, int, cudaStream_t);
 int* device_error_word();
 }  // namespace attn
 
@@ -79,6 +82,17 @@ int num_sms() {
 }
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+
+// Device address of the kernels' error word, looked up once per device.
+int* error_word_for_current_device() {
+  static int* cache[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[dev]) cache[dev] = attn::device_error_word();
+  return cache[dev];
+}
 
 struct SplitPlan {
   int nsplit;
@@ -169,6 +183,11 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.draft_block = mask_kind == ATTN_MASK_DRAFT_BLOCK ? draft_block : 1;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   p.q_tiles = (int)ceil_div(Lq, kBlockM);
+  const long long n_units = (long long)B * Hq * ((p.q_tiles + 1) / 2);
+  if (n_units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  p.n_units = (int)n_units;
+  p.err = error_word_for_current_device();
+  if (!p.err) return ATTN_ERR_CUDA;
 
   CUtensorMap tq, tk, tv;
   const uint64_t dq[3] = {(uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq};
@@ -176,10 +195,10 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   if (!encode_bf16(&tq, q, 3, dq) || !encode_bf16(&tk, k, 3, dk) || !encode_bf16(&tv, v, 3, dk))
     return ATTN_ERR_CUDA;
 
-  dim3 grid((unsigned)p.q_tiles, (unsigned)(B * Hq), 1);
+  const int grid = (int)(n_units < num_sms() ? n_units : num_sms());
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = d == 64 ? attn::launch_fwd<64, false>(tq, tk, tv, p, grid, st)
-                          : attn::launch_fwd<128, false>(tq, tk, tv, p, grid, st);
+  cudaError_t e = d == 64 ? attn::launch_prefill<64>(tq, tk, tv, p, grid, st)
+                          : attn::launch_prefill<128>(tq, tk, tv, p, grid, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

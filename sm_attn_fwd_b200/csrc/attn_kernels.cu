@@ -697,12 +697,6 @@ cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template cudaError_t launch_fwd<64, false>(const CUtensorMap&, const CUtensorMap&,
-                                           const CUtensorMap&, const FwdParams&, dim3,
-                                           cudaStream_t);
-template cudaError_t launch_fwd<128, false>(const CUtensorMap&, const CUtensorMap&,
-                                            const CUtensorMap&, const FwdParams&, dim3,
-                                            cudaStream_t);
 template cudaError_t launch_fwd<64, true>(const CUtensorMap&, const CUtensorMap&,
                                           const CUtensorMap&, const FwdParams&, dim3,
                                           cudaStream_t);

@@ -40,6 +40,8 @@ struct FwdParams {
   int nsplit;        // splits covering Lk_max
   int row_tiles;     // 128-row tiles per (b, kv head): ceil(group * Lq / 128)
   int q_tiles;       // prefill: ceil(Lq / 128)
+  int n_units;       // prefill: work units (pairs of query tiles x B*Hq)
+  int* err;          // device error word
 };
 
 }  // namespace attn

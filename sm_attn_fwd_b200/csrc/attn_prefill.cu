@@ -1,0 +1,749 @@
+// Prefill attention forward for sm_100a: persistent CTAs, two query tiles per
+// work unit.
+//
+// Method ("FlashAttention 2 原理与 PyTorch 实战", sections 一, 3.1, 3.2): query
+// tiles stream K/V tiles through shared memory; S = Q K^T, mask, online softmax
+// with a running max and sum, rescale of the accumulator, O += P V; O and the
+// log-sum-exp are written at the end and the N x N scores never reach HBM.
+// Masks: the mask_mod predicate of "FlexAttention 是什么，以及 DFlash2 之谜的完整
+// 侦破" (section 1: causal, sliding window, non-causal, document ids; section 3:
+// symmetric window, block-diffusion draft mask).
+//
+// B200 mapping.  A work unit is two adjacent 128-row query tiles (A and B) of
+// one (batch, head); both consume the same K/V tiles, so one TMA stream feeds
+// four tcgen05 MMAs per key tile (S_A, S_B, P_A V, P_B V).  384 threads:
+//   warpgroup 0   warp 0: builds each unit's tile schedule (EMPTY / PARTIAL /
+//                 FULL per key tile and query tile, in shared memory, double
+//                 buffered) and issues the TMA loads (Q_A, Q_B, K/V ring);
+//                 warp 1: allocates tensor memory, lane 0 issues every MMA;
+//                 registers lowered to 72 per thread.
+//   warpgroup 1   softmax of tile A (one query row per thread = TMEM lane);
+//   warpgroup 2   softmax of tile B; registers raised to 216 per thread.
+// While warpgroup 1 turns S_A into P_A, the tensor core computes S_B and P_B V,
+// and the other way round.  Tensor memory: S_A [0,128), S_B [128,256) with P
+// (bf16) written over the first 64 columns of each, O_A at 256, O_B at 256 + d.
+// A CTA walks its units in a snake order over units sorted heaviest first.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "attn_params.h"
+#include "ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kRegsLow = 72;    // warpgroup 0 (producer, MMA)
+constexpr int kRegsHigh = 216;  // softmax warpgroups: 72*128 + 2*216*128 = 168*384
+constexpr int kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+constexpr int kBitWords = kMaxKvTiles / 32;
+
+struct Sched {
+  int t_lo, t_hi;   // union of the two query tiles' candidate key tiles
+  int n[2];         // non-empty key tiles per query tile
+  int last[2];      // last non-empty key tile per query tile (-1: none)
+  int pad[2];
+  uint32_t empty[2][kBitWords];
+  uint32_t full[2][kBitWords];
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int kAtoms = D / 64;
+  static constexpr int kAtomBytes = 128 * 128;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kOffQ = 0;  // Q_A, Q_B
+  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kNumBars = 17 + 4 * kStages;  // see the barrier slots below
+  static constexpr int kOffMisc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
+  static constexpr int kOffSched = kOffMisc + 64;
+  static constexpr int kSmemBytes = kOffSched + 2 * (int)sizeof(Sched);
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+};
+
+struct Misc {
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Barrier slots (8 bytes each).  [2] = one per query tile (or per schedule buffer).
+enum : int {
+  kQFull = 0,        // [2] TMA -> MMA: Q_x landed
+  kQEmpty = 2,       // [2] MMA -> TMA: last S_x of the unit issued and done
+  kSFull = 4,        // [2] MMA -> softmax x: S_x ready
+  kPFull = 6,        // [2] softmax x (128 arrivals) -> MMA: P_x written, O_x rescaled
+  kODone = 8,        // [2] MMA -> softmax x: P_x V done
+  kOFree = 10,       // [2] softmax x (128) -> MMA: O_x read out, may be overwritten
+  kSchedFull = 12,   // [2] schedule builder -> MMA, softmax
+  kSchedEmpty = 14,  // [2] MMA + 8 softmax warps -> schedule builder
+  kDrain = 16,       // MMA: all MMAs done
+  kKvBase = 17,      // k_full[S], k_empty[S], v_full[S], v_empty[S]
+};
+
+struct Unit {
+  int b, hq, hkv, bh;
+  int q0[2];        // first query row of tile A / B
+  int rows[2];      // valid rows of tile A / B (0 if the tile is past Lq)
+  long long pos0[2];  // absolute position of row 0 of tile A / B
+};
+
+__device__ __forceinline__ long long floor_div_ll(long long a, long long b) {
+  return a >= 0 ? a / b : -((-a + b - 1) / b);
+}
+
+__device__ __forceinline__ void key_bounds(const FwdParams& p, long long pos, long long& lo,
+                                           long long& hi) {
+  lo = 0;
+  hi = (long long)p.Lk - 1;
+  if (p.mask_kind == kMaskCausal) {
+    hi = min(hi, pos);
+  } else if (p.mask_kind == kMaskDraftBlock) {
+    const long long bd = p.draft_block;
+    hi = min(hi, (floor_div_ll(pos, bd) + 1) * bd - 1);
+  }
+  if (p.window_l >= 0) lo = max(lo, pos - (long long)p.window_l);
+  if (p.window_r >= 0) hi = min(hi, pos + (long long)p.window_r);
+}
+
+__device__ __forceinline__ bool bit_get(const uint32_t* bits, int i) {
+  return (bits[i >> 5] >> (i & 31)) & 1u;
+}
+
+// The u-th unit (0 = heaviest): pairs of query tiles, last pair first.
+__device__ __forceinline__ void decode_unit(const FwdParams& p, int u, Unit& w) {
+  const int BH = p.B * p.Hq;
+  const int n_pairs = (p.q_tiles + 1) / 2;
+  const int pair = n_pairs - 1 - u / BH;
+  w.bh = u % BH;
+  w.b = w.bh / p.Hq;
+  w.hq = w.bh % p.Hq;
+  w.hkv = w.hq / p.group;
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    const int q0 = (2 * pair + x) * 128;
+    w.q0[x] = q0;
+    w.rows[x] = max(0, min(128, p.Lq - q0));
+    w.pos0[x] = (long long)p.Lk - p.Lq + q0;
+  }
+}
+
+// Unit handled by CTA `cta` in round `r` (snake order), or -1.
+__device__ __forceinline__ int unit_of(const FwdParams& p, int cta, int r) {
+  const int G = gridDim.x;
+  const int idx = r * G + ((r & 1) ? (G - 1 - cta) : cta);
+  return idx < p.n_units ? idx : -1;
+}
+
+// Whole warp: classify the key tiles of unit w into sched.
+__device__ void build_sched(const FwdParams& p, const Unit& w, Sched* s, int lane) {
+  long long lo_first[2], hi_first[2], lo_last[2], hi_last[2];
+  int t_lo = 0x7fffffff, t_hi = -1;
+  bool any[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    any[x] = false;
+    lo_first[x] = hi_last[x] = 0;
+    hi_first[x] = lo_last[x] = -1;
+    if (w.rows[x] > 0) {
+      key_bounds(p, w.pos0[x], lo_first[x], hi_first[x]);
+      key_bounds(p, w.pos0[x] + w.rows[x] - 1, lo_last[x], hi_last[x]);
+      if (hi_last[x] >= lo_first[x] && hi_last[x] >= 0) {
+        any[x] = true;
+        t_lo = min(t_lo, (int)(lo_first[x] / 128));
+        t_hi = max(t_hi, (int)(hi_last[x] / 128));
+      }
+    }
+  }
+  if (t_hi < 0) {
+    t_lo = 0;
+    t_hi = -1;
+  }
+  const int ntc = t_hi - t_lo + 1;
+  const int32_t* doc_b = p.doc_ids ? p.doc_ids + (long long)w.b * p.Lk : nullptr;
+  int qdmin[2] = {0, 0}, qdmax[2] = {0, 0};
+  if (doc_b) {
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      int mn = 0x7fffffff, mx = (int)0x80000000;
+      for (int r = lane; r < w.rows[x]; r += 32) {
+        const int d = __ldg(doc_b + (w.pos0[x] + r));
+        mn = min(mn, d);
+        mx = max(mx, d);
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      }
+      qdmin[x] = mn;
+      qdmax[x] = mx;
+    }
+  }
+  int cnt[2] = {0, 0}, last[2] = {-1, -1};
+  for (int base = 0; base < ntc; base += 32) {
+    const int i = base + lane;
+    const long long k0 = (long long)(t_lo + i) * 128;
+    bool empty[2], full[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      empty[x] = (i >= ntc) || !any[x] || k0 > hi_last[x] || k0 + 127 < lo_first[x];
+      full[x] = !empty[x] && (k0 + 128 <= p.Lk) && (lo_last[x] <= k0) &&
+                (hi_first[x] >= k0 + 127);
+    }
+    if (doc_b) {
+      for (int ww = 0; ww < 32 && base + ww < ntc; ++ww) {
+        const long long kb = (long long)(t_lo + base + ww) * 128;
+        const int kend = (int)min(kb + 128, (long long)p.Lk);
+        int mn = 0x7fffffff, mx = (int)0x80000000;
+        for (long long kk = kb + lane; kk < kend; kk += 32) {
+          const int d = __ldg(doc_b + kk);
+          mn = min(mn, d);
+          mx = max(mx, d);
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+          mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        if (lane == ww) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            if (mx < qdmin[x] || mn > qdmax[x]) empty[x] = true;
+            if (!(mn == mx && qdmin[x] == qdmax[x] && mn == qdmin[x])) full[x] = false;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      const uint32_t eb = __ballot_sync(0xffffffffu, empty[x]);
+      const uint32_t fb = __ballot_sync(0xffffffffu, full[x] && !empty[x]);
+      if (lane == 0) {
+        s->empty[x][base >> 5] = eb;
+        s->full[x][base >> 5] = fb;
+      }
+      cnt[x] += __popc(~eb);
+      if (~eb) last[x] = t_lo + base + 31 - __clz(~eb);
+    }
+  }
+  if (lane == 0) {
+    s->t_lo = t_lo;
+    s->t_hi = t_hi;
+    s->n[0] = cnt[0];
+    s->n[1] = cnt[1];
+    s->last[0] = last[0];
+    s->last[1] = last[1];
+  }
+}
+
+__device__ __forceinline__ bool tile_used(const Sched* s, int t) {
+  const int i = t - s->t_lo;
+  return !(bit_get(s->empty[0], i) && bit_get(s->empty[1], i));
+}
+
+// Shared-memory descriptors (128-byte swizzle, 1024-byte stride between 8-row
+// groups): the high word is the same for every operand here, the low word
+// holds the start address and the leading offset (16-byte units).
+constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+
+__device__ __forceinline__ uint64_t make_desc(uint32_t addr, uint32_t lbo_bytes) {
+  const uint32_t lo = ((addr >> 4) & 0x3FFFu) | ((lbo_bytes >> 4) << 16);
+  return ((uint64_t)kDescHi << 32) | lo;
+}
+
+template <int D>
+__device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int kk) {
+  return make_desc(tile_saddr + (kk >> 2) * Cfg<D>::kAtomBytes + (kk & 3) * 32, 16);
+}
+
+template <int D>
+__device__ __forceinline__ uint64_t desc_v(uint32_t tile_saddr, int kk) {
+  return make_desc(tile_saddr + kk * 2048, Cfg<D>::kAtomBytes);
+}
+
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_k,
+                        const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using C = Cfg<D>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  // 32-bit shared-memory addresses of the tiles and barriers
+  const uint32_t sq = ptx::smem_u32(smem + C::kOffQ);
+  const uint32_t sk = ptx::smem_u32(smem + C::kOffK);
+  const uint32_t sv_ = ptx::smem_u32(smem + C::kOffV);
+  const uint32_t bar0 = ptx::smem_u32(smem + C::kOffBar);
+  auto BAR = [bar0](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  Misc* misc = reinterpret_cast<Misc*>(smem + C::kOffMisc);
+  Sched* scheds = reinterpret_cast<Sched*>(smem + C::kOffSched);
+  volatile int* abort_flag = &misc->abort;
+  int* err = p.err;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int cta = blockIdx.x;
+
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    for (int x = 0; x < 2; ++x) {
+      ptx::mbar_init(&bars[kQFull + x], 1);
+      ptx::mbar_init(&bars[kQEmpty + x], 1);
+      ptx::mbar_init(&bars[kSFull + x], 1);
+      ptx::mbar_init(&bars[kPFull + x], 128);
+      ptx::mbar_init(&bars[kODone + x], 1);
+      ptx::mbar_init(&bars[kOFree + x], 128);
+      ptx::mbar_init(&bars[kSchedFull + x], 1);
+      ptx::mbar_init(&bars[kSchedEmpty + x], 1 + 8);
+    }
+    for (int st = 0; st < S; ++st) {
+      ptx::mbar_init(&bars[kKvBase + st], 1);          // k_full
+      ptx::mbar_init(&bars[kKvBase + S + st], 1);      // k_empty
+      ptx::mbar_init(&bars[kKvBase + 2 * S + st], 1);  // v_full
+      ptx::mbar_init(&bars[kKvBase + 3 * S + st], 1);  // v_empty
+    }
+    ptx::mbar_init(&bars[kDrain], 1);
+    misc->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(&misc->tmem_base, kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+  auto K_FULL = [&](int st) { return BAR(kKvBase + st); };
+  auto K_EMPTY = [&](int st) { return BAR(kKvBase + S + st); };
+  auto V_FULL = [&](int st) { return BAR(kKvBase + 2 * S + st); };
+  auto V_EMPTY = [&](int st) { return BAR(kKvBase + 3 * S + st); };
+
+  if (warp < 4) {
+    ptx::regs_dec<kRegsLow>();
+    if (warp == 0) {
+      // ---------------------------------------- schedule builder + TMA producer
+      int jkv = 0;
+      int rounds = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_of(p, cta, r);
+        if (u < 0) break;
+        rounds = r + 1;
+        Unit w;
+        decode_unit(p, u, w);
+        Sched* s = &scheds[r & 1];
+        ok = ptx::mbar_wait_a(BAR(kSchedEmpty + (r & 1)), (((uint32_t)r >> 1) & 1u) ^ 1u,
+                              abort_flag, err, kDevErrTimeoutProducer);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        build_sched(p, w, s, lane);
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive_a(BAR(kSchedFull + (r & 1)));
+          constexpr uint32_t kTx = C::kTileBytes;
+          for (int x = 0; x < 2 && ok; ++x) {
+            ok = ptx::mbar_wait_a(BAR(kQEmpty + x), ((uint32_t)r & 1u) ^ 1u, abort_flag, err,
+                                  kDevErrTimeoutProducer);
+            if (!ok) break;
+            ptx::mbar_arrive_expect_tx_a(BAR(kQFull + x), kTx);
+            for (int a = 0; a < C::kAtoms; ++a)
+              ptx::tma_load_3d_a(sq + x * C::kTileBytes + a * C::kAtomBytes, &tm_q,
+                                 BAR(kQFull + x), a * 64, w.q0[x], w.bh);
+          }
+          const int kv_z = w.b * p.Hkv + w.hkv;
+          const int t_hi = s->t_hi;
+          for (int t = s->t_lo; t <= t_hi && ok; ++t) {
+            if (!tile_used(s, t)) continue;
+            const int st = jkv % S;
+            const uint32_t ph = (uint32_t)(jkv / S) & 1u;
+            ok = ptx::mbar_wait_a(K_EMPTY(st), ph ^ 1u, abort_flag, err, kDevErrTimeoutProducer);
+            if (!ok) break;
+            ptx::mbar_arrive_expect_tx_a(K_FULL(st), kTx);
+            for (int a = 0; a < C::kAtoms; ++a)
+              ptx::tma_load_3d_a(sk + st * C::kTileBytes + a * C::kAtomBytes, &tm_k, K_FULL(st),
+                                 a * 64, t * 128, kv_z);
+            ok = ptx::mbar_wait_a(V_EMPTY(st), ph ^ 1u, abort_flag, err, kDevErrTimeoutProducer);
+            if (!ok) {
+              ++jkv;  // its K load is in flight: drain it below
+              break;
+            }
+            ptx::mbar_arrive_expect_tx_a(V_FULL(st), kTx);
+            for (int a = 0; a < C::kAtoms; ++a)
+              ptx::tma_load_3d_a(sv_ + st * C::kTileBytes + a * C::kAtomBytes, &tm_v, V_FULL(st),
+                                 a * 64, t * 128, kv_z);
+            ++jkv;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        jkv = __shfl_sync(0xffffffffu, jkv, 0);
+      }
+      // Drain: every TMA write into shared memory lands before the CTA exits
+      // (in a normal run these phases completed long ago).
+      if (lane == 0) {
+        int dummy = 0;
+        for (int jj = max(0, jkv - S); jj < jkv; ++jj) {
+          const uint32_t ph = (uint32_t)(jj / S) & 1u;
+          dummy = 0;
+          ptx::mbar_wait_a(K_FULL(jj % S), ph, &dummy, nullptr, 0);
+          dummy = 0;
+          ptx::mbar_wait_a(V_FULL(jj % S), ph, &dummy, nullptr, 0);
+        }
+        if (rounds > 0) {
+          for (int x = 0; x < 2; ++x) {
+            dummy = 0;
+            ptx::mbar_wait_a(BAR(kQFull + x), (uint32_t)(rounds - 1) & 1u, &dummy, nullptr, 0);
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, 0, 0);
+        constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, 0, 1);
+        int jkv = 0;
+        int ns0 = 0, ns1 = 0;  // S MMAs issued per query tile (global count)
+        bool ok = true;
+        for (int r = 0; ok; ++r) {
+          const int u = unit_of(p, cta, r);
+          if (u < 0) break;
+          const Sched* s = &scheds[r & 1];
+          ok = ptx::mbar_wait_a(BAR(kSchedFull + (r & 1)), ((uint32_t)r >> 1) & 1u, abort_flag,
+                                err, kDevErrTimeoutMma);
+          for (int x = 0; x < 2 && ok; ++x)
+            ok = ptx::mbar_wait_a(BAR(kQFull + x), (uint32_t)r & 1u, abort_flag, err,
+                                  kDevErrTimeoutMma);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          const int t_lo = s->t_lo, t_hi = s->t_hi;
+          const int last0 = s->last[0], last1 = s->last[1];
+          bool first0 = true, first1 = true;
+          // S_x(t) = Q_x K(t)^T into S_x; K(t) sits in stage st
+          auto issue_s = [&](int t, int st, int x) {
+            const uint32_t d_tmem = tmem + (x ? 128u : 0u);
+            const uint32_t qa = sq + x * C::kTileBytes;
+            const uint32_t ka = sk + st * C::kTileBytes;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              ptx::mma_ss(d_tmem, desc_kmajor<D>(qa, kk), desc_kmajor<D>(ka, kk), kIdescS,
+                          kk > 0 ? 1u : 0u);
+            ptx::mma_commit_a(BAR(kSFull + x));
+            if (x) ++ns1; else ++ns0;
+            if (t == (x ? last1 : last0)) ptx::mma_commit_a(BAR(kQEmpty + x));
+          };
+          int t = t_lo;
+          while (t <= t_hi && !tile_used(s, t)) ++t;
+          if (t <= t_hi) {
+            const int st = jkv % S;
+            ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+                                  kDevErrTimeoutMma);
+            if (ok) {
+              ptx::tc_fence_after();
+              for (int x = 0; x < 2; ++x)
+                if (!bit_get(s->empty[x], t - t_lo)) issue_s(t, st, x);
+              ptx::mma_commit_a(K_EMPTY(st));
+            }
+          }
+          while (ok && t <= t_hi) {
+            int tn = t + 1;
+            while (tn <= t_hi && !tile_used(s, tn)) ++tn;
+            const bool has_next = tn <= t_hi;
+            const int st = jkv % S;
+            const int stn = (jkv + 1) % S;
+            bool k_ready = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+              if (!bit_get(s->empty[x], t - t_lo)) {
+                // O_x free (first P V of the unit), P_x(t) written, V(t) landed
+                if ((x ? first1 : first0) && r > 0) {
+                  ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag, err,
+                                        kDevErrTimeoutMma);
+                  if (!ok) break;
+                }
+                ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)((x ? ns1 : ns0) - 1) & 1u,
+                                      abort_flag, err, kDevErrTimeoutMma);
+                if (!ok) break;
+                ok = ptx::mbar_wait_a(V_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+                                      kDevErrTimeoutMma);
+                if (!ok) break;
+                ptx::tc_fence_after();
+                const uint32_t p_tmem = tmem + (x ? 128u : 0u);
+                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
+                const uint32_t va = sv_ + st * C::kTileBytes;
+                const uint32_t acc0 = (x ? first1 : first0) ? 0u : 1u;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                  ptx::mma_ts(o_tmem, p_tmem + kk * 8, desc_v<D>(va, kk), kIdescPV,
+                              kk > 0 ? 1u : acc0);
+                ptx::mma_commit_a(BAR(kODone + x));
+                if (x) first1 = false; else first0 = false;
+              }
+              // S_x of the next key tile right behind this tile's P_x V
+              if (has_next && !bit_get(s->empty[x], tn - t_lo)) {
+                if (!k_ready) {
+                  ok = ptx::mbar_wait_a(K_FULL(stn), (uint32_t)((jkv + 1) / S) & 1u, abort_flag,
+                                        err, kDevErrTimeoutMma);
+                  if (!ok) break;
+                  ptx::tc_fence_after();
+                  k_ready = true;
+                }
+                issue_s(tn, stn, x);
+              }
+            }
+            if (!ok) break;
+            ptx::mma_commit_a(V_EMPTY(st));
+            if (has_next) ptx::mma_commit_a(K_EMPTY(stn));  // both S of the next tile issued
+            ++jkv;
+            t = tn;
+          }
+          // a query tile with no key tile at all still releases its Q buffer
+          if (last0 < 0) ptx::mma_commit_a(BAR(kQEmpty + 0));
+          if (last1 < 0) ptx::mma_commit_a(BAR(kQEmpty + 1));
+          ptx::mbar_arrive_a(BAR(kSchedEmpty + (r & 1)));
+        }
+        ptx::mma_commit_a(BAR(kDrain));
+        int dummy = 0;
+        ptx::mbar_wait_a(BAR(kDrain), 0, &dummy, nullptr, 0);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax
+    ptx::regs_inc<kRegsHigh>();
+    const int x = (warp - 4) >> 2;  // query tile A (0) or B (1)
+    const int quarter = warp & 3;
+    const int r_row = quarter * 32 + lane;
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t s_col = x ? 128u : 0u;
+    const uint32_t o_col = 256u + (uint32_t)(x * D);
+    const uint32_t bar_s_full = BAR(kSFull + x);
+    const uint32_t bar_p_full = BAR(kPFull + x);
+    const uint32_t bar_o_done = BAR(kODone + x);
+    const uint32_t bar_o_free = BAR(kOFree + x);
+    const float c = p.scale_log2;
+    int ns = 0;  // S tiles consumed (global count)
+    bool ok = true;
+    for (int r = 0; ok; ++r) {
+      const int u = unit_of(p, cta, r);
+      if (u < 0) break;
+      Unit w;
+      decode_unit(p, u, w);
+      const Sched* s = &scheds[r & 1];
+      ok = ptx::mbar_wait_a(BAR(kSchedFull + (r & 1)), ((uint32_t)r >> 1) & 1u, abort_flag, err,
+                            kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      const bool row_ok = r_row < w.rows[x];
+      int row_lo = 0, row_hi = -1;  // visible key range, clamped to [0, Lk-1]
+      int row_doc = 0;
+      const int32_t* doc_b = nullptr;
+      if (row_ok) {
+        const long long pos = w.pos0[x] + r_row;
+        long long lo, hi;
+        key_bounds(p, pos, lo, hi);
+        row_lo = (int)max(0LL, min(lo, (long long)p.Lk));
+        row_hi = (int)max(-1LL, min(hi, (long long)p.Lk - 1));
+        if (p.doc_ids != nullptr) {
+          doc_b = p.doc_ids + (long long)w.b * p.Lk;
+          row_doc = __ldg(doc_b + pos);
+        }
+      }
+      const int t_lo = s->t_lo, t_hi = s->t_hi;
+      const int n_mine = s->n[x];
+      float m_ref = -INFINITY;
+      float l = 0.0f;
+      int jl = 0;
+      for (int t = t_lo; t <= t_hi && ok; ++t) {
+        if (bit_get(s->empty[x], t - t_lo)) continue;
+        const bool full = bit_get(s->full[x], t - t_lo);
+        const int k0 = t * 128;
+        ok = ptx::mbar_wait_a(bar_s_full, (uint32_t)ns & 1u, abort_flag, err,
+                              kDevErrTimeoutSoftmax);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        float sv[128];
+        {
+          uint32_t raw[32];
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            ptx::tmem_ld32(t_row + s_col + cc * 32, raw);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(raw[i]);
+          }
+        }
+        if (!full) {
+          // visible keys of this row inside the tile: [lo_rel, hi_rel], and with
+          // document ids one visibility bit per key (dm0..dm3 = keys 0..127)
+          const int lo_rel = max(0, min(128, row_lo - k0));
+          const int hi_rel = max(-1, min(127, row_hi - k0));
+          uint32_t dm0 = ~0u, dm1 = ~0u, dm2 = ~0u, dm3 = ~0u;
+          if (doc_b != nullptr) {
+            const int32_t* dk = doc_b + k0;
+            const int kmax = min(128, p.Lk - k0);
+#pragma unroll 1
+            for (int g = 0; g < 4; ++g) {
+              uint32_t bits = 0;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int kk = g * 32 + i;
+                const int dv = (kk < kmax) ? __ldg(dk + kk) : ~row_doc;
+                bits |= (dv == row_doc ? 1u : 0u) << i;
+              }
+              if (g == 0) dm0 = bits;
+              else if (g == 1) dm1 = bits;
+              else if (g == 2) dm2 = bits;
+              else dm3 = bits;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            const uint32_t word = i < 32 ? dm0 : (i < 64 ? dm1 : (i < 96 ? dm2 : dm3));
+            const bool vis = (i >= lo_rel) && (i <= hi_rel) && ((word >> (i & 31)) & 1u);
+            sv[i] = vis ? sv[i] : -INFINITY;
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+        const float m_new = fmaxf(m_ref, mx * c);
+        const bool need = m_new > m_ref + kRescaleThreshold;
+        const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;
+        if (jl > 0 && __any_sync(0xffffffffu, need)) {
+          // O_x holds P V of the earlier tiles; that P V is complete (it was
+          // issued before the S just read), the wait only confirms it.
+          ok = ptx::mbar_wait_a(bar_o_done, (uint32_t)(ns - 1) & 1u, abort_flag, err,
+                                kDevErrTimeoutSoftmax);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ptx::tc_fence_after();
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t raw[32];
+            ptx::tmem_ld32(t_row + o_col + cc * 32, raw);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+            ptx::tmem_st32(t_row + o_col + cc * 32, raw);
+          }
+        }
+        if (need) {
+          l *= alpha;
+          m_ref = m_new;
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+        float rowsum = 0.0f;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ptx::ex2(fmaf(sv[h * 32 + 2 * i], c, -m_use));
+            const float p1 = ptx::ex2(fmaf(sv[h * 32 + 2 * i + 1], c, -m_use));
+            rowsum += p0 + p1;
+            packed[i] = ptx::pack_bf16x2(p0, p1);
+          }
+          ptx::tmem_st16(t_row + s_col + h * 16, packed);
+        }
+        l += rowsum;
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive_a(bar_p_full);
+        ++ns;
+        ++jl;
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_a(BAR(kSchedEmpty + (r & 1)));
+      ok = __all_sync(0xffffffffu, ok);
+      // ------------------------------------------------------------- epilogue
+      const bool have_o = ok && n_mine > 0 && jl == n_mine;
+      if (have_o) {
+        ok = ptx::mbar_wait_a(bar_o_done, (uint32_t)(ns - 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutSoftmax);
+        ok = __all_sync(0xffffffffu, ok);
+        ptx::tc_fence_after();
+      }
+      const bool have = have_o && ok && l > 0.0f;
+      const float inv_l = have ? 1.0f / l : 0.0f;
+      const float lse_row = have ? (m_ref + ptx::lg2(l)) * kLn2 : -INFINITY;
+      const long long out_row = (long long)w.bh * p.Lq + w.q0[x] + r_row;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t raw[32];
+        if (have_o && ok) {
+          ptx::tmem_ld32(t_row + o_col + cc * 32, raw);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) raw[i] = 0u;
+        }
+        if (row_ok) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + out_row * D + cc * 32;
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v4;
+            v4.x = ptx::pack_bf16x2(__uint_as_float(raw[i]) * inv_l,
+                                    __uint_as_float(raw[i + 1]) * inv_l);
+            v4.y = ptx::pack_bf16x2(__uint_as_float(raw[i + 2]) * inv_l,
+                                    __uint_as_float(raw[i + 3]) * inv_l);
+            v4.z = ptx::pack_bf16x2(__uint_as_float(raw[i + 4]) * inv_l,
+                                    __uint_as_float(raw[i + 5]) * inv_l);
+            v4.w = ptx::pack_bf16x2(__uint_as_float(raw[i + 6]) * inv_l,
+                                    __uint_as_float(raw[i + 7]) * inv_l);
+            *reinterpret_cast<uint4*>(dst + i) = v4;
+          }
+        }
+      }
+      if (row_ok) p.lse[out_row] = lse_row;
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_a(bar_o_free);
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const FwdParams& p, int grid, cudaStream_t stream) {
+  auto kern = attn_prefill_kernel<D>;
+  constexpr int smem = Cfg<D>::kSmemAlloc;
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_prefill<64>(const CUtensorMap&, const CUtensorMap&,
+                                        const CUtensorMap&, const FwdParams&, int, cudaStream_t);
+template cudaError_t launch_prefill<128>(const CUtensorMap&, const CUtensorMap&,
+                                         const CUtensorMap&, const FwdParams&, int, cudaStream_t);
+
+}  // namespace attn

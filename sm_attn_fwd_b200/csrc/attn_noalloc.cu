@@ -14,7 +14,7 @@
 #include <cstdint>
 #include <mutex>
 
-#include "../../include/attn.h"
+#include "attn.h"
 
 namespace {
 

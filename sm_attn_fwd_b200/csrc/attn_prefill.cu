@@ -20,14 +20,17 @@
 //   warpgroup 1   softmax of tile A (one query row per thread = TMEM lane);
 //   warpgroup 2   softmax of tile B; registers raised to 216 per thread.
 // While warpgroup 1 turns S_A into P_A, the tensor core computes S_B and P_B V,
-// and the other way round.  Tensor memory: S_A [0,128), S_B [128,256) with P
-// (bf16) written over the first 64 columns of each, O_A at 256, O_B at 256 + d.
+// and the other way round.  Tensor memory: S_A [0,128), S_B [128,256), O_A at
+// 256, O_B at 256 + d.  P (bf16, 64 columns) is written over S when d = 128;
+// when d = 64 it has columns of its own ([384,448), [448,512)), so the next
+// key tile's S_x is computed while the softmax still works on this one.
 // A CTA walks its units in a snake order over units sorted heaviest first.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "attn_params.h"
 #include "ptx.cuh"
@@ -62,7 +65,11 @@ struct Cfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 17 + 4 * kStages;  // see the barrier slots below
+  static constexpr int kNumBars = 19 + 4 * kStages;  // see the barrier slots below
+  // d = 64 leaves tensor-memory columns for P of its own ([384,448) and
+  // [448,512)), so S_x of the next key tile can be computed while the softmax
+  // still works on this one; d = 128 writes P over S.
+  static constexpr bool kSepP = (D == 64);
   static constexpr int kOffMisc = kOffBar + ((kNumBars * 8 + 15) / 16) * 16;
   static constexpr int kOffSched = kOffMisc + 64;
   static constexpr int kSmemBytes = kOffSched + 2 * (int)sizeof(Sched);
@@ -85,7 +92,8 @@ enum : int {
   kSchedFull = 12,   // [2] schedule builder -> MMA, softmax
   kSchedEmpty = 14,  // [2] MMA + 8 softmax warps -> schedule builder
   kDrain = 16,       // MMA: all MMAs done
-  kKvBase = 17,      // k_full[S], k_empty[S], v_full[S], v_empty[S]
+  kSFree = 17,       // [2] softmax x (128) -> MMA: S_x loaded into registers (separate-P mode)
+  kKvBase = 19,      // k_full[S], k_empty[S], v_full[S], v_empty[S]
 };
 
 struct Unit {
@@ -112,6 +120,31 @@ __device__ __forceinline__ void key_bounds(const FwdParams& p, long long pos, lo
   if (p.window_l >= 0) lo = max(lo, pos - (long long)p.window_l);
   if (p.window_r >= 0) hi = min(hi, pos + (long long)p.window_r);
 }
+
+// exp2 on the FMA pipe, to take part of the exponentials off the MUFU unit:
+// x = n + r with n = round(x) (the 1.5 * 2^23 trick), r in [-1/2, 1/2];
+// 2^r ~ q(r) = 1 + r*(c1 + r*(c2 + r*c3)), coefficients from
+// csrc/gen_exp2_poly.py (minimax relative error 1.0e-4 with q(0) = 1, so
+// integer arguments are exact); 2^n is added to the exponent field.  x is
+// clamped at -126, so the result is never exactly 0: only tiles without
+// masked keys use it.
+__device__ __forceinline__ float exp2_fma(float x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x = fmaxf(x, -126.0f);
+  const float t = x + kRound;
+  const float r = x - (t - kRound);
+  float q = fmaf(5.500893295e-02f, r, 2.422109544e-01f);
+  q = fmaf(q, r, 6.932829022e-01f);
+  q = fmaf(q, r, 1.0f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
+// Which of the 128 exponentials of a row go to the FMA pipe.  Measured on
+// B200 (causal 4K d=64 and 32K d=128): any share made the kernel slower
+// (1/8: -4%, 2/8: -7%), since the softmax is bound by instruction issue and
+// handoff latency, not by the MUFU unit; kept switched off.
+constexpr bool kExpFmaShare = false;
+__host__ __device__ constexpr bool exp_on_fma(int i) { return (i & 7) == 3 && kExpFmaShare; }
 
 __device__ __forceinline__ bool bit_get(const uint32_t* bits, int i) {
   return (bits[i >> 5] >> (i & 31)) & 1u;
@@ -308,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars[kOFree + x], 128);
       ptx::mbar_init(&bars[kSchedFull + x], 1);
       ptx::mbar_init(&bars[kSchedEmpty + x], 1 + 8);
+      ptx::mbar_init(&bars[kSFree + x], 128);
     }
     for (int st = 0; st < S; ++st) {
       ptx::mbar_init(&bars[kKvBase + st], 1);          // k_full
@@ -411,11 +445,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
-      if (lane == 0) {
+      // The whole warp runs this loop with warp-uniform values; elect.sync
+      // picks the lane that issues each tcgen05.mma / commit.
+      {
         constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, 0, 0);
         constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, 0, 1);
         int jkv = 0;
         int ns0 = 0, ns1 = 0;  // S MMAs issued per query tile (global count)
+        int np0 = 0, np1 = 0;  // P V MMAs issued per query tile (separate-P mode)
         bool ok = true;
         for (int r = 0; ok; ++r) {
           const int u = unit_of(p, cta, r);
@@ -426,6 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int x = 0; x < 2 && ok; ++x)
             ok = ptx::mbar_wait_a(BAR(kQFull + x), (uint32_t)r & 1u, abort_flag, err,
                                   kDevErrTimeoutMma);
+          ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ptx::tc_fence_after();
           const int t_lo = s->t_lo, t_hi = s->t_hi;
@@ -434,86 +472,149 @@ __global__ void __launch_bounds__(kThreads, 1)
           // S_x(t) = Q_x K(t)^T into S_x; K(t) sits in stage st
           auto issue_s = [&](int t, int st, int x) {
             const uint32_t d_tmem = tmem + (x ? 128u : 0u);
-            const uint32_t qa = sq + x * C::kTileBytes;
-            const uint32_t ka = sk + st * C::kTileBytes;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk)
-              ptx::mma_ss(d_tmem, desc_kmajor<D>(qa, kk), desc_kmajor<D>(ka, kk), kIdescS,
-                          kk > 0 ? 1u : 0u);
-            ptx::mma_commit_a(BAR(kSFull + x));
+            const uint64_t qd = desc_kmajor<D>(sq + x * C::kTileBytes, 0);
+            const uint64_t kd = desc_kmajor<D>(sk + st * C::kTileBytes, 0);
+            if constexpr (D == 64)
+              ptx::mma_qk_chain_d64(d_tmem, qd, kd, kIdescS);
+            else
+              ptx::mma_qk_chain_d128(d_tmem, qd, kd, kIdescS);
+            ptx::mma_commit_warp(BAR(kSFull + x));
             if (x) ++ns1; else ++ns0;
-            if (t == (x ? last1 : last0)) ptx::mma_commit_a(BAR(kQEmpty + x));
+            if (t == (x ? last1 : last0)) ptx::mma_commit_warp(BAR(kQEmpty + x));
           };
-          int t = t_lo;
-          while (t <= t_hi && !tile_used(s, t)) ++t;
-          if (t <= t_hi) {
-            const int st = jkv % S;
-            ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
-                                  kDevErrTimeoutMma);
-            if (ok) {
-              ptx::tc_fence_after();
-              for (int x = 0; x < 2; ++x)
-                if (!bit_get(s->empty[x], t - t_lo)) issue_s(t, st, x);
-              ptx::mma_commit_a(K_EMPTY(st));
-            }
-          }
-          while (ok && t <= t_hi) {
-            int tn = t + 1;
-            while (tn <= t_hi && !tile_used(s, tn)) ++tn;
-            const bool has_next = tn <= t_hi;
-            const int st = jkv % S;
-            const int stn = (jkv + 1) % S;
-            bool k_ready = false;
-            for (int x = 0; x < 2 && ok; ++x) {
-              if (!bit_get(s->empty[x], t - t_lo)) {
-                // O_x free (first P V of the unit), P_x(t) written, V(t) landed
-                if ((x ? first1 : first0) && r > 0) {
-                  ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag, err,
+          if constexpr (C::kSepP) {
+            // Separate P: S_x of key tile t is issued as soon as the softmax has
+            // loaded S_x of the previous tile; P_x V of that previous tile goes
+            // right after, when P_x is written.
+            int t_prev = -1, j_prev = 0;
+            auto issue_pv = [&](int tp, int jp) -> bool {
+              const int stp = jp % S;
+              for (int x = 0; x < 2; ++x) {
+                if (bit_get(s->empty[x], tp - t_lo)) continue;
+                bool w_ok = true;
+                if ((x ? first1 : first0) && r > 0)
+                  w_ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag,
+                                          err, kDevErrTimeoutMma);
+                if (w_ok)
+                  w_ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)(x ? np1 : np0) & 1u,
+                                          abort_flag, err, kDevErrTimeoutMma);
+                if (w_ok)
+                  w_ok = ptx::mbar_wait_a(V_FULL(stp), (uint32_t)(jp / S) & 1u, abort_flag, err,
+                                          kDevErrTimeoutMma);
+                if (!__all_sync(0xffffffffu, w_ok)) return false;
+                ptx::tc_fence_after();
+                const uint32_t p_tmem = tmem + 384u + (uint32_t)(x * 64);
+                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
+                const uint32_t acc0 = (x ? first1 : first0) ? 0u : 1u;
+                ptx::mma_pv_chain8(o_tmem, p_tmem, desc_v<D>(sv_ + stp * C::kTileBytes, 0),
+                                   kIdescPV, acc0);
+                ptx::mma_commit_warp(BAR(kODone + x));
+                if (x) { first1 = false; ++np1; } else { first0 = false; ++np0; }
+              }
+              ptx::mma_commit_warp(V_EMPTY(stp));
+              return true;
+            };
+            for (int t = t_lo; t <= t_hi && ok; ++t) {
+              if (!tile_used(s, t)) continue;
+              const int st = jkv % S;
+              bool k_ready = false;
+              for (int x = 0; x < 2 && ok; ++x) {
+                if (bit_get(s->empty[x], t - t_lo)) continue;
+                // the softmax has loaded S_x of its previous tile
+                if ((x ? ns1 : ns0) > 0)
+                  ok = ptx::mbar_wait_a(BAR(kSFree + x), (uint32_t)((x ? ns1 : ns0) - 1) & 1u,
+                                        abort_flag, err, kDevErrTimeoutMma);
+                if (ok && !k_ready)
+                  ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
                                         kDevErrTimeoutMma);
-                  if (!ok) break;
-                }
-                ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)((x ? ns1 : ns0) - 1) & 1u,
-                                      abort_flag, err, kDevErrTimeoutMma);
-                if (!ok) break;
-                ok = ptx::mbar_wait_a(V_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
-                                      kDevErrTimeoutMma);
+                ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                const uint32_t p_tmem = tmem + (x ? 128u : 0u);
-                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
-                const uint32_t va = sv_ + st * C::kTileBytes;
-                const uint32_t acc0 = (x ? first1 : first0) ? 0u : 1u;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                  ptx::mma_ts(o_tmem, p_tmem + kk * 8, desc_v<D>(va, kk), kIdescPV,
-                              kk > 0 ? 1u : acc0);
-                ptx::mma_commit_a(BAR(kODone + x));
-                if (x) first1 = false; else first0 = false;
+                k_ready = true;
+                issue_s(t, st, x);
               }
-              // S_x of the next key tile right behind this tile's P_x V
-              if (has_next && !bit_get(s->empty[x], tn - t_lo)) {
-                if (!k_ready) {
-                  ok = ptx::mbar_wait_a(K_FULL(stn), (uint32_t)((jkv + 1) / S) & 1u, abort_flag,
-                                        err, kDevErrTimeoutMma);
-                  if (!ok) break;
-                  ptx::tc_fence_after();
-                  k_ready = true;
-                }
-                issue_s(tn, stn, x);
+              if (!ok) break;
+              ptx::mma_commit_warp(K_EMPTY(st));
+              if (t_prev >= 0) ok = issue_pv(t_prev, j_prev);
+              t_prev = t;
+              j_prev = jkv;
+              ++jkv;
+            }
+            if (ok && t_prev >= 0) ok = issue_pv(t_prev, j_prev);
+          } else {
+            int t = t_lo;
+            while (t <= t_hi && !tile_used(s, t)) ++t;
+            if (t <= t_hi) {
+              const int st = jkv % S;
+              ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+                                    kDevErrTimeoutMma);
+              ok = __all_sync(0xffffffffu, ok);
+              if (ok) {
+                ptx::tc_fence_after();
+                for (int x = 0; x < 2; ++x)
+                  if (!bit_get(s->empty[x], t - t_lo)) issue_s(t, st, x);
+                ptx::mma_commit_warp(K_EMPTY(st));
               }
             }
-            if (!ok) break;
-            ptx::mma_commit_a(V_EMPTY(st));
-            if (has_next) ptx::mma_commit_a(K_EMPTY(stn));  // both S of the next tile issued
-            ++jkv;
-            t = tn;
+            while (ok && t <= t_hi) {
+              int tn = t + 1;
+              while (tn <= t_hi && !tile_used(s, tn)) ++tn;
+              const bool has_next = tn <= t_hi;
+              const int st = jkv % S;
+              const int stn = (jkv + 1) % S;
+              bool k_ready = false;
+              for (int x = 0; x < 2 && ok; ++x) {
+                if (!bit_get(s->empty[x], t - t_lo)) {
+                  // O_x free (first P V of the unit), P_x(t) written, V(t) landed
+                  if ((x ? first1 : first0) && r > 0) {
+                    ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag, err,
+                                          kDevErrTimeoutMma);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                  }
+                  ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)((x ? ns1 : ns0) - 1) & 1u,
+                                        abort_flag, err, kDevErrTimeoutMma);
+                  ok = __all_sync(0xffffffffu, ok);
+                  if (!ok) break;
+                  ok = ptx::mbar_wait_a(V_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+                                        kDevErrTimeoutMma);
+                  ok = __all_sync(0xffffffffu, ok);
+                  if (!ok) break;
+                  ptx::tc_fence_after();
+                  const uint32_t p_tmem = tmem + (x ? 128u : 0u);
+                  const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
+                  const uint32_t va = sv_ + st * C::kTileBytes;
+                  const uint32_t acc0 = (x ? first1 : first0) ? 0u : 1u;
+                  ptx::mma_pv_chain8(o_tmem, p_tmem, desc_v<D>(va, 0), kIdescPV, acc0);
+                  ptx::mma_commit_warp(BAR(kODone + x));
+                  if (x) first1 = false; else first0 = false;
+                }
+                // S_x of the next key tile right behind this tile's P_x V
+                if (has_next && !bit_get(s->empty[x], tn - t_lo)) {
+                  if (!k_ready) {
+                    ok = ptx::mbar_wait_a(K_FULL(stn), (uint32_t)((jkv + 1) / S) & 1u, abort_flag,
+                                          err, kDevErrTimeoutMma);
+                    ok = __all_sync(0xffffffffu, ok);
+                    if (!ok) break;
+                    ptx::tc_fence_after();
+                    k_ready = true;
+                  }
+                  issue_s(tn, stn, x);
+                }
+              }
+              if (!ok) break;
+              ptx::mma_commit_warp(V_EMPTY(st));
+              if (has_next) ptx::mma_commit_warp(K_EMPTY(stn));  // both S of the next tile issued
+              ++jkv;
+              t = tn;
+            }
           }
           // a query tile with no key tile at all still releases its Q buffer
-          if (last0 < 0) ptx::mma_commit_a(BAR(kQEmpty + 0));
-          if (last1 < 0) ptx::mma_commit_a(BAR(kQEmpty + 1));
-          ptx::mbar_arrive_a(BAR(kSchedEmpty + (r & 1)));
+          if (last0 < 0) ptx::mma_commit_warp(BAR(kQEmpty + 0));
+          if (last1 < 0) ptx::mma_commit_warp(BAR(kQEmpty + 1));
+          if (lane == 0) ptx::mbar_arrive_a(BAR(kSchedEmpty + (r & 1)));
         }
-        ptx::mma_commit_a(BAR(kDrain));
+        ptx::mma_commit_warp(BAR(kDrain));
         int dummy = 0;
         ptx::mbar_wait_a(BAR(kDrain), 0, &dummy, nullptr, 0);
       }
@@ -527,6 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
     const uint32_t s_col = x ? 128u : 0u;
     const uint32_t o_col = 256u + (uint32_t)(x * D);
+    const uint32_t p_col = C::kSepP ? 384u + (uint32_t)(x * 64) : s_col;
     const uint32_t bar_s_full = BAR(kSFull + x);
     const uint32_t bar_p_full = BAR(kPFull + x);
     const uint32_t bar_o_done = BAR(kODone + x);
@@ -575,13 +677,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tc_fence_after();
         float sv[128];
         {
-          uint32_t raw[32];
+          // all four 32-column loads in flight, one wait
+          uint32_t r0[32], r1[32], r2[32], r3[32];
+          ptx::tmem_ld32(t_row + s_col + 0, r0);
+          ptx::tmem_ld32(t_row + s_col + 32, r1);
+          ptx::tmem_ld32(t_row + s_col + 64, r2);
+          ptx::tmem_ld32(t_row + s_col + 96, r3);
+          ptx::tmem_wait_ld();
+          if constexpr (C::kSepP) {
+            // S_x is in registers: its columns may take the next tile's S_x
+            ptx::tc_fence_before();
+            ptx::mbar_arrive_a(BAR(kSFree + x));
+          }
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            ptx::tmem_ld32(t_row + s_col + cc * 32, raw);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) sv[cc * 32 + i] = __uint_as_float(raw[i]);
+          for (int i = 0; i < 32; ++i) {
+            sv[i] = __uint_as_float(r0[i]);
+            sv[32 + i] = __uint_as_float(r1[i]);
+            sv[64 + i] = __uint_as_float(r2[i]);
+            sv[96 + i] = __uint_as_float(r3[i]);
           }
         }
         if (!full) {
@@ -615,20 +728,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[i] = vis ? sv[i] : -INFINITY;
           }
         }
-        float mx = -INFINITY;
+        // row max with eight independent chains, then a tree
+        float mx8[8];
 #pragma unroll
-        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, sv[i]);
+        for (int j = 0; j < 8; ++j) mx8[j] = sv[j];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) mx8[j] = fmaxf(mx8[j], mx8[j + 4]);
+        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
         const float m_new = fmaxf(m_ref, mx * c);
         const bool need = m_new > m_ref + kRescaleThreshold;
         const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;
-        if (jl > 0 && __any_sync(0xffffffffu, need)) {
-          // O_x holds P V of the earlier tiles; that P V is complete (it was
-          // issued before the S just read), the wait only confirms it.
+        if (C::kSepP && jl > 0) {
+          // P_x V of the previous tile must be done before P_x is overwritten
+          // (and before O_x is rescaled)
           ok = ptx::mbar_wait_a(bar_o_done, (uint32_t)(ns - 1) & 1u, abort_flag, err,
                                 kDevErrTimeoutSoftmax);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ptx::tc_fence_after();
+        }
+        if (jl > 0 && __any_sync(0xffffffffu, need)) {
+          // O_x holds P V of the earlier tiles; with P over S that P V is
+          // complete (it was issued before the S just read): the wait confirms it.
+          if constexpr (!C::kSepP) {
+            ok = ptx::mbar_wait_a(bar_o_done, (uint32_t)(ns - 1) & 1u, abort_flag, err,
+                                  kDevErrTimeoutSoftmax);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) break;
+            ptx::tc_fence_after();
+          }
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t raw[32];
@@ -645,20 +775,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_ref = m_new;
         }
         const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-        float rowsum = 0.0f;
+        float sum8[8];
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t packed[16];
+        for (int j = 0; j < 8; ++j) sum8[j] = 0.0f;
+        // P = 2^(s*c - m), bf16, written over S; FULL tiles send a quarter of
+        // the exponentials to the FMA pipe, PARTIAL tiles keep exact zeros.
+        auto emit_p = [&](auto fma_share) {
+          constexpr bool kShare = decltype(fma_share)::value;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ptx::ex2(fmaf(sv[h * 32 + 2 * i], c, -m_use));
-            const float p1 = ptx::ex2(fmaf(sv[h * 32 + 2 * i + 1], c, -m_use));
-            rowsum += p0 + p1;
-            packed[i] = ptx::pack_bf16x2(p0, p1);
+          for (int h = 0; h < 4; ++h) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int i0 = h * 32 + 2 * i, i1 = i0 + 1;
+              const float a0 = fmaf(sv[i0], c, -m_use);
+              const float a1 = fmaf(sv[i1], c, -m_use);
+              const float p0 = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
+              const float p1 = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
+              sum8[i0 & 7] += p0;
+              sum8[i1 & 7] += p1;
+              packed[i] = ptx::pack_bf16x2(p0, p1);
+            }
+            ptx::tmem_st16(t_row + p_col + h * 16, packed);
           }
-          ptx::tmem_st16(t_row + s_col + h * 16, packed);
-        }
-        l += rowsum;
+        };
+        if (full)
+          emit_p(std::true_type{});
+        else
+          emit_p(std::false_type{});
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sum8[j] += sum8[j + 4];
+        l += (sum8[0] + sum8[1]) + (sum8[2] + sum8[3]);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive_a(bar_p_full);

@@ -65,7 +65,7 @@ struct Cfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 19 + 4 * kStages;  // see the barrier slots below
+  static constexpr int kNumBars = 21 + 4 * kStages;  // see the barrier slots below
   // d = 64 leaves tensor-memory columns for P of its own ([384,448) and
   // [448,512)), so S_x of the next key tile can be computed while the softmax
   // still works on this one; d = 128 writes P over S.
@@ -93,7 +93,8 @@ enum : int {
   kSchedEmpty = 14,  // [2] MMA + 8 softmax warps -> schedule builder
   kDrain = 16,       // MMA: all MMAs done
   kSFree = 17,       // [2] softmax x (128) -> MMA: S_x loaded into registers (separate-P mode)
-  kKvBase = 19,      // k_full[S], k_empty[S], v_full[S], v_empty[S]
+  kTurn = 19,        // [2] softmax 1-x (128) -> softmax x: x may run its exponentials
+  kKvBase = 21,      // k_full[S], k_empty[S], v_full[S], v_empty[S]
 };
 
 struct Unit {
@@ -342,6 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars[kSchedFull + x], 1);
       ptx::mbar_init(&bars[kSchedEmpty + x], 1 + 8);
       ptx::mbar_init(&bars[kSFree + x], 128);
+      ptx::mbar_init(&bars[kTurn + x], 128);
     }
     for (int st = 0; st < S; ++st) {
       ptx::mbar_init(&bars[kKvBase + st], 1);          // k_full
@@ -635,6 +637,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_o_free = BAR(kOFree + x);
     const float c = p.scale_log2;
     int ns = 0;  // S tiles consumed (global count)
+    // The two softmax warpgroups take turns on the exponentials of each key
+    // tile (A, B, A, B, ...), so that one loads S, finds the row max and stores
+    // P while the other keeps the MUFU unit busy.  kTurn[x] completes once per
+    // turn handed to x; B hands A the first turn.
+    const uint32_t bar_my_turn = BAR(kTurn + x);
+    const uint32_t bar_other_turn = BAR(kTurn + (x ^ 1));
+    int turns = 0;
+    if (x == 1) ptx::mbar_arrive_a(bar_other_turn);
     bool ok = true;
     for (int r = 0; ok; ++r) {
       const int u = unit_of(p, cta, r);
@@ -667,7 +677,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.0f;
       int jl = 0;
       for (int t = t_lo; t <= t_hi && ok; ++t) {
-        if (bit_get(s->empty[x], t - t_lo)) continue;
+        if (!tile_used(s, t)) continue;
+        if (bit_get(s->empty[x], t - t_lo)) {
+          // no key tile of ours here: pass the turn on
+          ok = ptx::mbar_wait_a(bar_my_turn, (uint32_t)turns & 1u, abort_flag, err,
+                                kDevErrTimeoutSoftmax);
+          ok = __all_sync(0xffffffffu, ok);
+          ++turns;
+          ptx::mbar_arrive_a(bar_other_turn);
+          continue;
+        }
         const bool full = bit_get(s->full[x], t - t_lo);
         const int k0 = t * 128;
         ok = ptx::mbar_wait_a(bar_s_full, (uint32_t)ns & 1u, abort_flag, err,
@@ -740,25 +759,56 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_new = fmaxf(m_ref, mx * c);
         const bool need = m_new > m_ref + kRescaleThreshold;
         const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;
-        if (C::kSepP && jl > 0) {
-          // P_x V of the previous tile must be done before P_x is overwritten
-          // (and before O_x is rescaled)
+        if (need) {
+          l *= alpha;
+          m_ref = m_new;
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+        // P = 2^(s*c - m) as packed bf16 pairs, all in registers first, so the
+        // wait for the previous P V (below) overlaps the exponentials.
+        uint32_t pk[64];
+        float sum8[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sum8[j] = 0.0f;
+        auto emit_p = [&](auto fma_share) {
+          constexpr bool kShare = decltype(fma_share)::value;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int i0 = 2 * i, i1 = i0 + 1;
+            const float a0 = fmaf(sv[i0], c, -m_use);
+            const float a1 = fmaf(sv[i1], c, -m_use);
+            const float p0 = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
+            const float p1 = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
+            sum8[i0 & 7] += p0;
+            sum8[i1 & 7] += p1;
+            pk[i] = ptx::pack_bf16x2(p0, p1);
+          }
+        };
+        ok = ptx::mbar_wait_a(bar_my_turn, (uint32_t)turns & 1u, abort_flag, err,
+                              kDevErrTimeoutSoftmax);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++turns;
+        if (full)
+          emit_p(std::true_type{});  // FULL tiles may send exponentials to the FMA pipe
+        else
+          emit_p(std::false_type{});  // PARTIAL tiles keep exact zeros at masked keys
+        ptx::mbar_arrive_a(bar_other_turn);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sum8[j] += sum8[j + 4];
+        l += (sum8[0] + sum8[1]) + (sum8[2] + sum8[3]);
+        // P_x V of the previous tile must be done before O_x is rescaled and,
+        // with separate P columns, before P_x is overwritten.  With P over S it
+        // is already done (it was issued before the S just read).
+        const bool any_need = __any_sync(0xffffffffu, need);
+        if (jl > 0 && (C::kSepP || any_need)) {
           ok = ptx::mbar_wait_a(bar_o_done, (uint32_t)(ns - 1) & 1u, abort_flag, err,
                                 kDevErrTimeoutSoftmax);
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           ptx::tc_fence_after();
         }
-        if (jl > 0 && __any_sync(0xffffffffu, need)) {
-          // O_x holds P V of the earlier tiles; with P over S that P V is
-          // complete (it was issued before the S just read): the wait confirms it.
-          if constexpr (!C::kSepP) {
-            ok = ptx::mbar_wait_a(bar_o_done, (uint32_t)(ns - 1) & 1u, abort_flag, err,
-                                  kDevErrTimeoutSoftmax);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) break;
-            ptx::tc_fence_after();
-          }
+        if (jl > 0 && any_need) {
 #pragma unroll
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t raw[32];
@@ -770,42 +820,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_st32(t_row + o_col + cc * 32, raw);
           }
         }
-        if (need) {
-          l *= alpha;
-          m_ref = m_new;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          uint32_t chunk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) chunk[i] = pk[h * 16 + i];
+          ptx::tmem_st16(t_row + p_col + h * 16, chunk);
         }
-        const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-        float sum8[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) sum8[j] = 0.0f;
-        // P = 2^(s*c - m), bf16, written over S; FULL tiles send a quarter of
-        // the exponentials to the FMA pipe, PARTIAL tiles keep exact zeros.
-        auto emit_p = [&](auto fma_share) {
-          constexpr bool kShare = decltype(fma_share)::value;
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            uint32_t packed[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int i0 = h * 32 + 2 * i, i1 = i0 + 1;
-              const float a0 = fmaf(sv[i0], c, -m_use);
-              const float a1 = fmaf(sv[i1], c, -m_use);
-              const float p0 = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
-              const float p1 = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
-              sum8[i0 & 7] += p0;
-              sum8[i1 & 7] += p1;
-              packed[i] = ptx::pack_bf16x2(p0, p1);
-            }
-            ptx::tmem_st16(t_row + p_col + h * 16, packed);
-          }
-        };
-        if (full)
-          emit_p(std::true_type{});
-        else
-          emit_p(std::false_type{});
-#pragma unroll
-        for (int j = 0; j < 4; ++j) sum8[j] += sum8[j + 4];
-        l += (sum8[0] + sum8[1]) + (sum8[2] + sum8[3]);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive_a(bar_p_full);

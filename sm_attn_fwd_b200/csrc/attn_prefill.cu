@@ -310,6 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = Cfg<D>;
   constexpr int S = C::kStages;
+  constexpr int kMmaWarps = C::kSepP ? 2 : 1;  // warps issuing MMAs
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -341,17 +342,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars[kODone + x], 1);
       ptx::mbar_init(&bars[kOFree + x], 128);
       ptx::mbar_init(&bars[kSchedFull + x], 1);
-      ptx::mbar_init(&bars[kSchedEmpty + x], 1 + 8);
+      ptx::mbar_init(&bars[kSchedEmpty + x], kMmaWarps + 8);
       ptx::mbar_init(&bars[kSFree + x], 128);
       ptx::mbar_init(&bars[kTurn + x], 128);
     }
     for (int st = 0; st < S; ++st) {
       ptx::mbar_init(&bars[kKvBase + st], 1);          // k_full
-      ptx::mbar_init(&bars[kKvBase + S + st], 1);      // k_empty
+      ptx::mbar_init(&bars[kKvBase + S + st], kMmaWarps);      // k_empty
       ptx::mbar_init(&bars[kKvBase + 2 * S + st], 1);  // v_full
-      ptx::mbar_init(&bars[kKvBase + 3 * S + st], 1);  // v_empty
+      ptx::mbar_init(&bars[kKvBase + 3 * S + st], kMmaWarps);  // v_empty
     }
-    ptx::mbar_init(&bars[kDrain], 1);
+    ptx::mbar_init(&bars[kDrain], kMmaWarps);
     misc->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -445,7 +446,101 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-    } else if (warp == 1) {
+    } else if (C::kSepP && (warp == 1 || warp == 2)) {
+      // ------------------------------------ MMA issuers, d = 64: one per query tile
+      // Warp 1 issues every MMA of query tile A and warp 2 those of tile B, so
+      // neither waits on the other tile's softmax.  With separate P columns,
+      // S_x of key tile t only needs the softmax to have loaded the previous
+      // S_x, and P_x V of the previous tile follows when P_x is written.  Both
+      // warps release every K/V stage (two arrivals), each after that stage's
+      // load has landed, so the ring's phases stay in order.
+      const int x = warp - 1;
+      constexpr uint32_t kIdescS = ptx::idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t d_tmem = tmem + (x ? 128u : 0u);
+      const uint32_t p_tmem = tmem + 384u + (uint32_t)(x * 64);
+      const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
+      const uint64_t q_desc = desc_kmajor<D>(sq + x * C::kTileBytes, 0);
+      int jkv = 0, ns = 0, np = 0;
+      bool ok = true;
+      for (int r = 0; ok; ++r) {
+        const int u = unit_of(p, cta, r);
+        if (u < 0) break;
+        const Sched* s = &scheds[r & 1];
+        ok = ptx::mbar_wait_a(BAR(kSchedFull + (r & 1)), ((uint32_t)r >> 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutMma);
+        if (ok)
+          ok = ptx::mbar_wait_a(BAR(kQFull + x), (uint32_t)r & 1u, abort_flag, err,
+                                kDevErrTimeoutMma);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const int t_lo = s->t_lo, t_hi = s->t_hi;
+        const int last = s->last[x];
+        bool first = true;
+        // P_x V of key tile tp (union index jp), then release its V stage
+        auto issue_pv = [&](int tp, int jp) -> bool {
+          const int stp = jp % S;
+          const bool mine = !bit_get(s->empty[x], tp - t_lo);
+          bool w_ok = ptx::mbar_wait_a(V_FULL(stp), (uint32_t)(jp / S) & 1u, abort_flag, err,
+                                       kDevErrTimeoutMma);
+          if (w_ok && mine && first && r > 0)
+            w_ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag, err,
+                                    kDevErrTimeoutMma);
+          if (w_ok && mine)
+            w_ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)np & 1u, abort_flag, err,
+                                    kDevErrTimeoutMma);
+          if (!__all_sync(0xffffffffu, w_ok)) return false;
+          ptx::tc_fence_after();
+          if (mine) {
+            ptx::mma_pv_chain8(o_tmem, p_tmem, desc_v<D>(sv_ + stp * C::kTileBytes, 0), kIdescPV,
+                               first ? 0u : 1u);
+            ptx::mma_commit_warp(BAR(kODone + x));
+            ++np;
+            first = false;
+          }
+          ptx::mma_commit_warp(V_EMPTY(stp));
+          return true;
+        };
+        int t_prev = -1, j_prev = 0;
+        for (int t = t_lo; t <= t_hi && ok; ++t) {
+          if (!tile_used(s, t)) continue;
+          const int st = jkv % S;
+          const bool mine = !bit_get(s->empty[x], t - t_lo);
+          // the softmax has loaded the previous S_x; K(t) has landed
+          if (mine && ns > 0)
+            ok = ptx::mbar_wait_a(BAR(kSFree + x), (uint32_t)(ns - 1) & 1u, abort_flag, err,
+                                  kDevErrTimeoutMma);
+          if (ok)
+            ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+                                  kDevErrTimeoutMma);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          if (mine) {
+            const uint64_t k_desc = desc_kmajor<D>(sk + st * C::kTileBytes, 0);
+            if constexpr (D == 64)
+              ptx::mma_qk_chain_d64(d_tmem, q_desc, k_desc, kIdescS);
+            else
+              ptx::mma_qk_chain_d128(d_tmem, q_desc, k_desc, kIdescS);
+            ptx::mma_commit_warp(BAR(kSFull + x));
+            ++ns;
+            if (t == last) ptx::mma_commit_warp(BAR(kQEmpty + x));  // Q_x no longer read
+          }
+          ptx::mma_commit_warp(K_EMPTY(st));
+          if (t_prev >= 0) ok = issue_pv(t_prev, j_prev);
+          t_prev = t;
+          j_prev = jkv;
+          ++jkv;
+        }
+        if (ok && t_prev >= 0) ok = issue_pv(t_prev, j_prev);
+        if (last < 0) ptx::mma_commit_warp(BAR(kQEmpty + x));  // no key tile: Q_x unused
+        if (lane == 0) ptx::mbar_arrive_a(BAR(kSchedEmpty + (r & 1)));
+      }
+      ptx::mma_commit_warp(BAR(kDrain));
+      int dummy = 0;
+      ptx::mbar_wait_a(BAR(kDrain), 0, &dummy, nullptr, 0);
+    } else if (!C::kSepP && warp == 1) {
       // ---------------------------------------------------------- MMA issuer
       // The whole warp runs this loop with warp-uniform values; elect.sync
       // picks the lane that issues each tcgen05.mma / commit.
@@ -454,7 +549,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t kIdescPV = ptx::idesc_bf16_f32(128, D, 0, 1);
         int jkv = 0;
         int ns0 = 0, ns1 = 0;  // S MMAs issued per query tile (global count)
-        int np0 = 0, np1 = 0;  // P V MMAs issued per query tile (separate-P mode)
         bool ok = true;
         for (int r = 0; ok; ++r) {
           const int u = unit_of(p, cta, r);
@@ -484,132 +578,71 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (x) ++ns1; else ++ns0;
             if (t == (x ? last1 : last0)) ptx::mma_commit_warp(BAR(kQEmpty + x));
           };
-          if constexpr (C::kSepP) {
-            // Separate P: S_x of key tile t is issued as soon as the softmax has
-            // loaded S_x of the previous tile; P_x V of that previous tile goes
-            // right after, when P_x is written.
-            int t_prev = -1, j_prev = 0;
-            auto issue_pv = [&](int tp, int jp) -> bool {
-              const int stp = jp % S;
-              for (int x = 0; x < 2; ++x) {
-                if (bit_get(s->empty[x], tp - t_lo)) continue;
-                bool w_ok = true;
-                if ((x ? first1 : first0) && r > 0)
-                  w_ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag,
-                                          err, kDevErrTimeoutMma);
-                if (w_ok)
-                  w_ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)(x ? np1 : np0) & 1u,
-                                          abort_flag, err, kDevErrTimeoutMma);
-                if (w_ok)
-                  w_ok = ptx::mbar_wait_a(V_FULL(stp), (uint32_t)(jp / S) & 1u, abort_flag, err,
-                                          kDevErrTimeoutMma);
-                if (!__all_sync(0xffffffffu, w_ok)) return false;
-                ptx::tc_fence_after();
-                const uint32_t p_tmem = tmem + 384u + (uint32_t)(x * 64);
-                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
-                const uint32_t acc0 = (x ? first1 : first0) ? 0u : 1u;
-                ptx::mma_pv_chain8(o_tmem, p_tmem, desc_v<D>(sv_ + stp * C::kTileBytes, 0),
-                                   kIdescPV, acc0);
-                ptx::mma_commit_warp(BAR(kODone + x));
-                if (x) { first1 = false; ++np1; } else { first0 = false; ++np0; }
-              }
-              ptx::mma_commit_warp(V_EMPTY(stp));
-              return true;
-            };
-            for (int t = t_lo; t <= t_hi && ok; ++t) {
-              if (!tile_used(s, t)) continue;
-              const int st = jkv % S;
-              bool k_ready = false;
-              for (int x = 0; x < 2 && ok; ++x) {
-                if (bit_get(s->empty[x], t - t_lo)) continue;
-                // the softmax has loaded S_x of its previous tile
-                if ((x ? ns1 : ns0) > 0)
-                  ok = ptx::mbar_wait_a(BAR(kSFree + x), (uint32_t)((x ? ns1 : ns0) - 1) & 1u,
-                                        abort_flag, err, kDevErrTimeoutMma);
-                if (ok && !k_ready)
-                  ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+          int t = t_lo;
+          while (t <= t_hi && !tile_used(s, t)) ++t;
+          if (t <= t_hi) {
+            const int st = jkv % S;
+            ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+                                  kDevErrTimeoutMma);
+            ok = __all_sync(0xffffffffu, ok);
+            if (ok) {
+              ptx::tc_fence_after();
+              for (int x = 0; x < 2; ++x)
+                if (!bit_get(s->empty[x], t - t_lo)) issue_s(t, st, x);
+              ptx::mma_commit_warp(K_EMPTY(st));
+            }
+          }
+          while (ok && t <= t_hi) {
+            int tn = t + 1;
+            while (tn <= t_hi && !tile_used(s, tn)) ++tn;
+            const bool has_next = tn <= t_hi;
+            const int st = jkv % S;
+            const int stn = (jkv + 1) % S;
+            bool k_ready = false;
+            for (int x = 0; x < 2 && ok; ++x) {
+              if (!bit_get(s->empty[x], t - t_lo)) {
+                // O_x free (first P V of the unit), P_x(t) written, V(t) landed
+                if ((x ? first1 : first0) && r > 0) {
+                  ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag, err,
                                         kDevErrTimeoutMma);
+                  ok = __all_sync(0xffffffffu, ok);
+                  if (!ok) break;
+                }
+                ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)((x ? ns1 : ns0) - 1) & 1u,
+                                      abort_flag, err, kDevErrTimeoutMma);
+                ok = __all_sync(0xffffffffu, ok);
+                if (!ok) break;
+                ok = ptx::mbar_wait_a(V_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
+                                      kDevErrTimeoutMma);
                 ok = __all_sync(0xffffffffu, ok);
                 if (!ok) break;
                 ptx::tc_fence_after();
-                k_ready = true;
-                issue_s(t, st, x);
+                const uint32_t p_tmem = tmem + (x ? 128u : 0u);
+                const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
+                const uint32_t va = sv_ + st * C::kTileBytes;
+                const uint32_t acc0 = (x ? first1 : first0) ? 0u : 1u;
+                ptx::mma_pv_chain8(o_tmem, p_tmem, desc_v<D>(va, 0), kIdescPV, acc0);
+                ptx::mma_commit_warp(BAR(kODone + x));
+                if (x) first1 = false; else first0 = false;
               }
-              if (!ok) break;
-              ptx::mma_commit_warp(K_EMPTY(st));
-              if (t_prev >= 0) ok = issue_pv(t_prev, j_prev);
-              t_prev = t;
-              j_prev = jkv;
-              ++jkv;
-            }
-            if (ok && t_prev >= 0) ok = issue_pv(t_prev, j_prev);
-          } else {
-            int t = t_lo;
-            while (t <= t_hi && !tile_used(s, t)) ++t;
-            if (t <= t_hi) {
-              const int st = jkv % S;
-              ok = ptx::mbar_wait_a(K_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
-                                    kDevErrTimeoutMma);
-              ok = __all_sync(0xffffffffu, ok);
-              if (ok) {
-                ptx::tc_fence_after();
-                for (int x = 0; x < 2; ++x)
-                  if (!bit_get(s->empty[x], t - t_lo)) issue_s(t, st, x);
-                ptx::mma_commit_warp(K_EMPTY(st));
-              }
-            }
-            while (ok && t <= t_hi) {
-              int tn = t + 1;
-              while (tn <= t_hi && !tile_used(s, tn)) ++tn;
-              const bool has_next = tn <= t_hi;
-              const int st = jkv % S;
-              const int stn = (jkv + 1) % S;
-              bool k_ready = false;
-              for (int x = 0; x < 2 && ok; ++x) {
-                if (!bit_get(s->empty[x], t - t_lo)) {
-                  // O_x free (first P V of the unit), P_x(t) written, V(t) landed
-                  if ((x ? first1 : first0) && r > 0) {
-                    ok = ptx::mbar_wait_a(BAR(kOFree + x), (uint32_t)(r - 1) & 1u, abort_flag, err,
-                                          kDevErrTimeoutMma);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                  }
-                  ok = ptx::mbar_wait_a(BAR(kPFull + x), (uint32_t)((x ? ns1 : ns0) - 1) & 1u,
-                                        abort_flag, err, kDevErrTimeoutMma);
-                  ok = __all_sync(0xffffffffu, ok);
-                  if (!ok) break;
-                  ok = ptx::mbar_wait_a(V_FULL(st), (uint32_t)(jkv / S) & 1u, abort_flag, err,
-                                        kDevErrTimeoutMma);
+              // S_x of the next key tile right behind this tile's P_x V
+              if (has_next && !bit_get(s->empty[x], tn - t_lo)) {
+                if (!k_ready) {
+                  ok = ptx::mbar_wait_a(K_FULL(stn), (uint32_t)((jkv + 1) / S) & 1u, abort_flag,
+                                        err, kDevErrTimeoutMma);
                   ok = __all_sync(0xffffffffu, ok);
                   if (!ok) break;
                   ptx::tc_fence_after();
-                  const uint32_t p_tmem = tmem + (x ? 128u : 0u);
-                  const uint32_t o_tmem = tmem + 256u + (uint32_t)(x * D);
-                  const uint32_t va = sv_ + st * C::kTileBytes;
-                  const uint32_t acc0 = (x ? first1 : first0) ? 0u : 1u;
-                  ptx::mma_pv_chain8(o_tmem, p_tmem, desc_v<D>(va, 0), kIdescPV, acc0);
-                  ptx::mma_commit_warp(BAR(kODone + x));
-                  if (x) first1 = false; else first0 = false;
+                  k_ready = true;
                 }
-                // S_x of the next key tile right behind this tile's P_x V
-                if (has_next && !bit_get(s->empty[x], tn - t_lo)) {
-                  if (!k_ready) {
-                    ok = ptx::mbar_wait_a(K_FULL(stn), (uint32_t)((jkv + 1) / S) & 1u, abort_flag,
-                                          err, kDevErrTimeoutMma);
-                    ok = __all_sync(0xffffffffu, ok);
-                    if (!ok) break;
-                    ptx::tc_fence_after();
-                    k_ready = true;
-                  }
-                  issue_s(tn, stn, x);
-                }
+                issue_s(tn, stn, x);
               }
-              if (!ok) break;
-              ptx::mma_commit_warp(V_EMPTY(st));
-              if (has_next) ptx::mma_commit_warp(K_EMPTY(stn));  // both S of the next tile issued
-              ++jkv;
-              t = tn;
             }
+            if (!ok) break;
+            ptx::mma_commit_warp(V_EMPTY(st));
+            if (has_next) ptx::mma_commit_warp(K_EMPTY(stn));  // both S of the next tile issued
+            ++jkv;
+            t = tn;
           }
           // a query tile with no key tile at all still releases its Q buffer
           if (last0 < 0) ptx::mma_commit_warp(BAR(kQEmpty + 0));

@@ -780,15 +780,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[i] = vis ? sv[i] : -INFINITY;
           }
         }
-        // row max with eight independent chains, then a tree
+        // row max: eight independent chains of three-input max, then a tree
         float mx8[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) mx8[j] = sv[j];
+        for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(sv[j], sv[8 + j]);
 #pragma unroll
-        for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], sv[i]);
+        for (int i = 16; i < 128; i += 16) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) mx8[j] = fmaxf(mx8[j], mx8[j + 4]);
-        const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3]));
+          for (int j = 0; j < 8; ++j) mx8[j] = ptx::max3(mx8[j], sv[i + j], sv[i + 8 + j]);
+        }
+        const float mx = fmaxf(ptx::max3(mx8[0], mx8[1], mx8[2]),
+                               ptx::max3(mx8[3], ptx::max3(mx8[4], mx8[5], mx8[6]), mx8[7]));
         const float m_new = fmaxf(m_ref, mx * c);
         const bool need = m_new > m_ref + kRescaleThreshold;
         const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;
@@ -799,8 +801,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
         // P = 2^(s*c - m) as packed bf16 pairs, all in registers first, so the
         // wait for the previous P V (below) overlaps the exponentials.
-        uint32_t pk[64];
-        float sum8[8];
+        // four 16-column pieces, each the register range of one tcgen05.st
+        uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
+        float sum8[8];  // four packed (even, odd) partial sums
 #pragma unroll
         for (int j = 0; j < 8; ++j) sum8[j] = 0.0f;
         auto emit_p = [&](auto fma_share) {
@@ -808,13 +811,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
             const int i0 = 2 * i, i1 = i0 + 1;
-            const float a0 = fmaf(sv[i0], c, -m_use);
-            const float a1 = fmaf(sv[i1], c, -m_use);
+            float a0, a1;
+            ptx::fma2_bc(a0, a1, sv[i0], sv[i1], c, -m_use);  // s * c - m, two at once
             const float p0 = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
             const float p1 = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
-            sum8[i0 & 7] += p0;
-            sum8[i1 & 7] += p1;
-            pk[i] = ptx::pack_bf16x2(p0, p1);
+            ptx::add2_acc(sum8[(i & 3) * 2], sum8[(i & 3) * 2 + 1], p0, p1);
+            const uint32_t packed = ptx::pack_bf16x2(p0, p1);
+            if (i < 16) pk0[i] = packed;
+            else if (i < 32) pk1[i - 16] = packed;
+            else if (i < 48) pk2[i - 32] = packed;
+            else pk3[i - 48] = packed;
           }
         };
         ok = ptx::mbar_wait_a(bar_my_turn, (uint32_t)turns & 1u, abort_flag, err,
@@ -853,13 +859,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tmem_st32(t_row + o_col + cc * 32, raw);
           }
         }
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          uint32_t chunk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) chunk[i] = pk[h * 16 + i];
-          ptx::tmem_st16(t_row + p_col + h * 16, chunk);
-        }
+        ptx::tmem_st16(t_row + p_col + 0, pk0);
+        ptx::tmem_st16(t_row + p_col + 16, pk1);
+        ptx::tmem_st16(t_row + p_col + 32, pk2);
+        ptx::tmem_st16(t_row + p_col + 48, pk3);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive_a(bar_p_full);

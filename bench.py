@@ -168,10 +168,15 @@ def profiled_traffic():
     summary, or None when the kernel sources changed since that capture."""
     try:
         from sm_attn_fwd_b200 import build as _build
-        with open(os.path.join(ROOT, "profiles", "attn_fwd_causal4k_traffic.json")) as f:
-            rec = json.load(f)
-        if rec.get("kernel_digest") == _build.source_digest():
-            return float(rec["dram_bytes_per_launch"])
+        fields = {}
+        with open(os.path.join(ROOT, "profiles", "attn_prefill_causal4k_d64.md")) as f:
+            for line in f:
+                if ":" in line and line.split(":", 1)[0] in ("kernel_digest",
+                                                             "traffic_bytes_per_launch"):
+                    k, v = line.split(":", 1)
+                    fields[k] = v.strip()
+        if fields.get("kernel_digest") == _build.source_digest():
+            return float(fields["traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
         pass
     return None
@@ -469,7 +474,7 @@ def main():
             "roofline": {"bound": "tensor", "achieved": per_launch_tflops,
                          "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": per_launch_tflops / peaks["bf16_tflops"],
-                         "traffic": profiled_traffic(), "kernel": "attn_fwd_kernel<64,false>",
+                         "traffic": profiled_traffic(), "kernel": "attn_prefill_kernel<64>",
                          "algorithmic_flop_per_launch": flops,
                          "peak_source": f"{peaks['source']} bf16_tflops (burst)"},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,

@@ -188,6 +188,17 @@ attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* k_cache,
  */
 attn_status_t attn_get_device_error(void* stream, int* raw_bits);
 
+/*
+ * attn_selftest_wait_timeout — diagnostic for the failure-detection path (no
+ * counterpart on the pages).  Enqueues on `stream` a one-block kernel whose
+ * single bounded wait targets an mbarrier that nothing arrives on: the wait
+ * gives up after its budget (about one second), records the self-test timeout
+ * bit in the device error word and returns.  A following
+ * attn_get_device_error() returns ATTN_ERR_TIMEOUT and clears the word; the
+ * CUDA context stays usable.  Returns ATTN_ERR_CUDA if the launch fails.
+ */
+attn_status_t attn_selftest_wait_timeout(void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* attn_status_string(attn_status_t s);
 

@@ -27,7 +27,7 @@ __all__ = [
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
     "attn_fwd", "attn_decode_splitkv", "attn_decode_num_splits",
     "attn_decode_workspace_size", "attn_decode_splitkv_noalloc", "attn_get_device_error",
-    "attn_status_string",
+    "attn_selftest_wait_timeout", "attn_status_string",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -46,7 +46,7 @@ _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 EXPORTED_SYMBOLS = (
     "attn_fwd", "attn_decode_num_splits", "attn_decode_workspace_size",
     "attn_decode_splitkv", "attn_decode_splitkv_noalloc", "attn_get_device_error",
-    "attn_status_string",
+    "attn_selftest_wait_timeout", "attn_status_string",
 )
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -91,6 +91,8 @@ def load_library():
         lib.attn_decode_splitkv_noalloc.restype = i32
         lib.attn_get_device_error.argtypes = [P, ctypes.POINTER(ctypes.c_int)]
         lib.attn_get_device_error.restype = i32
+        lib.attn_selftest_wait_timeout.argtypes = [P]
+        lib.attn_selftest_wait_timeout.restype = i32
         lib.attn_status_string.argtypes = [i32]
         lib.attn_status_string.restype = ctypes.c_char_p
         _lib = lib
@@ -222,6 +224,14 @@ def attn_decode_splitkv_noalloc(q, k_cache, v_cache, kv_lens, *, scale=None, num
     if st != ATTN_OK:
         raise AttnError(st, "attn_decode_splitkv_noalloc")
     return o, lse
+
+
+def attn_selftest_wait_timeout(stream=None):
+    """Enqueue the failure-detection self-test kernel (see include/attn.h)."""
+    dev = torch.cuda.current_device()
+    st = load_library().attn_selftest_wait_timeout(_stream_handle(stream, dev))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_wait_timeout")
 
 
 def attn_get_device_error(stream=None):

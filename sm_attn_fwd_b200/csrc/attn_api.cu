@@ -23,6 +23,7 @@ template <int D>
 cudaError_t launch_prefill(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                            const FwdParams&, int, cudaStream_t);
 int* device_error_word();
+cudaError_t launch_selftest_wait(cudaStream_t stream);
 }  // namespace attn
 
 namespace {
@@ -290,10 +291,15 @@ attn_status_t attn_get_device_error(void* stream, int* raw_bits) {
     return ATTN_ERR_CUDA;
   if (raw_bits) *raw_bits = bits;
   if (bits & (attn::kDevErrTimeoutProducer | attn::kDevErrTimeoutMma |
-              attn::kDevErrTimeoutSoftmax))
+              attn::kDevErrTimeoutSoftmax | attn::kDevErrTimeoutSelftest))
     return ATTN_ERR_TIMEOUT;
   if (bits & attn::kDevErrBadKvLen) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
+}
+
+attn_status_t attn_selftest_wait_timeout(void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return attn::launch_selftest_wait(st) == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -666,6 +666,31 @@ __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const FwdParam
   if (lane == 0) p.lse[row] = sum > 0.0f ? mx + ptx::lg2(sum) * kLn2 : -INFINITY;
 }
 
+// Failure-detection self-test: one thread waits, with the same bounded wait the
+// attention kernels use, on an mbarrier that nothing ever arrives on.  The wait
+// must give up after its budget, record kDevErrTimeoutSelftest and return, so
+// the host sees ATTN_ERR_TIMEOUT and the context stays usable.
+__global__ void attn_selftest_wait_kernel() {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const bool ok = ptx::mbar_wait_a(ptx::smem_u32(&bar), 0, &abort_flag, &g_device_error,
+                                     kDevErrTimeoutSelftest);
+    if (ok) atomicOr(&g_device_error, kDevErrBadKvLen);  // cannot happen: nobody arrives
+  }
+}
+
+cudaError_t launch_selftest_wait(cudaStream_t stream) {
+  attn_selftest_wait_kernel<<<1, 32, 0, stream>>>();
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------- launchers
 template <int D, bool kDecode>
 cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

@@ -18,6 +18,7 @@ enum DeviceError : int {
   kDevErrTimeoutMma = 1 << 1,
   kDevErrTimeoutSoftmax = 1 << 2,
   kDevErrBadKvLen = 1 << 3,
+  kDevErrTimeoutSelftest = 1 << 4,
 };
 
 struct FwdParams {

@@ -132,3 +132,24 @@ def test_config_decode_sampled(cfg):
         ro, rl = oracle.attn_fwd(qs, ks, vs, scale=cfg.softmax_scale)
         compare(o[b:b + 1, h * G:(h + 1) * G], lse[b:b + 1, h * G:(h + 1) * G], ro, rl,
                 f"{cfg.name} b={b} h={h}")
+
+
+def test_decode_capturable_in_cuda_graph():
+    q, k, v, _, kv = random_case(61, 2, 16, 2, 1, 900, 128, kv_len_range=(100, 900))
+    qd, kd, vd, kl = to_dev(q, k, v, kv)
+    ws = torch.empty(ab.attn_decode_workspace_size(2, 16, 2, 1, 900, 128), dtype=torch.uint8,
+                     device="cuda")
+    o = torch.empty_like(qd)
+    lse = torch.empty(2, 16, 1, dtype=torch.float32, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ab.attn_decode_splitkv(qd, kd, vd, kl, workspace=ws, o=o, lse=lse, stream=s)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        ab.attn_decode_splitkv(qd, kd, vd, kl, workspace=ws, o=o, lse=lse, stream=s)
+    o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    ro, rl = oracle.attn_fwd(q, k, v, kv_lens=kv)
+    compare(o, lse, ro, rl, "decode graph")

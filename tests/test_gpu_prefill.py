@@ -47,13 +47,20 @@ RAGGED = [
     (10, 1, 2, 2, 600, 200, 64, "causal", (-1, -1), 1, False),   # Lq > Lk: empty rows
     (11, 1, 2, 2, 130, 1000, 128, "draft", (3, 200), 7, False),
     (12, 1, 8, 2, 256, 1024, 64, "causal", (-1, -1), 1, False),
+    (13, 1, 16, 2, 1, 5000, 128, "causal", (-1, -1), 1, False),  # one query row
+    (14, 2, 8, 1, 700, 1900, 128, "none", (-1, -1), 1, False),    # GQA 8, Lq < Lk
+    (15, 1, 4, 4, 1000, 1000, 64, "causal", (-1, -1), 1, True),   # many documents
+    (16, 1, 2, 2, 900, 900, 128, "draft", (70, 33), 48, True),    # block not a divisor of 128
+    (17, 1, 2, 1, 383, 1150, 64, "causal", (200, 5), 1, False),   # causal + window, offset
+    (18, 3, 3, 3, 129, 129, 128, "none", (0, 0), 1, False),       # each row sees one key
 ]
 
 
 @pytest.mark.parametrize("case", RAGGED, ids=lambda c: f"s{c[0]}_{c[7]}_lq{c[4]}_lk{c[5]}_d{c[6]}")
 def test_ragged_shapes_and_masks(case):
     seed, B, Hq, Hkv, Lq, Lk, d, mask, window, bd, doc = case
-    q, k, v, doc_ids, _ = random_case(seed, B, Hq, Hkv, Lq, Lk, d, doc_split=doc, n_docs=3)
+    q, k, v, doc_ids, _ = random_case(seed, B, Hq, Hkv, Lq, Lk, d, doc_split=doc,
+                                      n_docs=8 if seed == 15 else 3)
     kw = dict(scale=1.0 / math.sqrt(d), mask=mask, window=window, draft_block=bd)
     o, lse = _run(q, k, v, doc_ids=doc_ids, **kw)
     ro, rl = oracle.attn_fwd(q, k, v, doc_ids=doc_ids, **kw)
@@ -175,3 +182,13 @@ def test_capturable_in_cuda_graph():
     torch.cuda.synchronize()
     ro, rl = oracle.attn_fwd(q, k, v, mask="causal")
     compare(o, lse, ro, rl, "graph")
+
+
+def test_repeated_calls_are_bit_identical():
+    """The persistent schedule is static: the same inputs give the same bits."""
+    q, k, v, _, _ = random_case(19, 2, 4, 2, 777, 777, 64)
+    qd, kd, vd = to_dev(q, k, v)
+    o1, l1 = ab.attn_fwd(qd, kd, vd, mask="causal")
+    o2, l2 = ab.attn_fwd(qd, kd, vd, mask="causal")
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)

@@ -247,6 +247,40 @@ def run_decode(cfg, timer, steps, warmup, stream):
     return inp, ms, decode_bytes(cfg, kv), (nsplit, chunk)
 
 
+def run_decode_paged(cfg, page_size, timer, steps, warmup, stream):
+    """The decode workload with its cache moved into a shuffled page pool
+    [num_pages, Hkv, page_size, d] addressed through a block table."""
+    import sm_attn_fwd_b200 as ab
+    inp = make_inputs(cfg, device="cuda")
+    B, Hkv, L, d = inp.k.shape
+    pps = L // page_size
+    g = torch.Generator(device="cuda")
+    g.manual_seed(cfg.seed + 1000)
+    perm = torch.randperm(B * pps, generator=g, device="cuda")
+    # logical page (b, i) goes to physical page perm[b * pps + i]
+    def to_pool(x):
+        pages = x.view(B, Hkv, pps, page_size, d).permute(0, 2, 1, 3, 4).reshape(B * pps, Hkv,
+                                                                                   page_size, d)
+        pool = torch.empty_like(pages)
+        pool[perm] = pages
+        return pool
+    kp, vp = to_pool(inp.k), to_pool(inp.v)
+    table = perm.view(B, pps).to(torch.int32).contiguous()
+    del inp.k, inp.v
+    torch.cuda.synchronize()
+    ws = torch.empty(ab.attn_decode_workspace_size(cfg.B, cfg.Hq, cfg.Hkv, cfg.Lq, cfg.Lk, cfg.d),
+                     dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(inp.q)
+    lse = torch.empty(cfg.B, cfg.Hq, cfg.Lq, dtype=torch.float32, device="cuda")
+    fn = lambda: ab.attn_decode_paged(inp.q, kp, vp, table, inp.kv_lens, scale=cfg.softmax_scale,  # noqa: E731
+                                      workspace=ws, o=o, lse=lse, stream=stream)
+    ms = timer.time(fn, steps, warmup)
+    st, bits = ab.attn_get_device_error(stream)
+    if st != ab.ATTN_OK:
+        raise RuntimeError(f"device error after paged {cfg.name}: {st} {bits}")
+    return ms, decode_bytes(cfg, inp.kv_lens.cpu().numpy())
+
+
 def e2e_prefill(cfg, steps, warmup, stream):
     """Same call with host buffers: H2D of Q, K, V, the kernel, D2H of O and LSE."""
     import sm_attn_fwd_b200 as ab
@@ -443,6 +477,15 @@ def main():
                                       "frac_of_8TBs_nominal": gbs / 8000.0,
                                       "algorithmic_bytes": nb, "splits": plan[0],
                                       "chunk_keys": plan[1]}
+            for psz in (128, 16):
+                ms4, nb4 = run_decode_paged(DECODE_LQ1, psz, timer, max(5, args.steps // 10), 3,
+                                            stream)
+                med = statistics.median(ms4)
+                gbs = nb4 / (med * 1e6)
+                workloads[f"{DECODE_LQ1.name}_paged{psz}"] = {
+                    "ms_median": med, "ms_min": min(ms4), "GB/s": gbs,
+                    "frac_of_hbm": gbs / peaks["hbm_gbs"], "algorithmic_bytes": nb4,
+                    "page_size": psz}
     torch.cuda.synchronize()
     barrier(world)
     clk = clocks.summary()

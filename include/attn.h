@@ -148,6 +148,39 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
                                   void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_decode_paged — the split-KV decode of attn_decode_splitkv over a paged
+ * KV cache (the paged block_table call of "FlexAttention 是什么，以及 DFlash2 之谜
+ * 的完整侦破", section 4, experiment 1; PagedAttention through a logical-to-
+ * physical page table, section 1).
+ *
+ * Defines: sequence b's logical key j lives in page block_table[b][j / page_size]
+ * at row j % page_size; the visible keys are [0, kv_lens[b]); O and LSE as in
+ * attn_decode_splitkv.  Equals attn_decode_splitkv on the cache gathered
+ * through the block table.
+ *
+ * Arguments
+ *   q                 [B, Hq, Lq, d] bf16
+ *   k_pages, v_pages  [num_pages, Hkv, page_size, d] bf16 page pool, read
+ *   block_table       [B, pages_per_seq] int32 DEVICE array of page ids in
+ *                     [0, num_pages); entries past a sequence's last page are
+ *                     never read; an out-of-range id reads as zeros and flags
+ *                     the device error word (ATTN_ERR_INVALID_ARG)
+ *   o, lse, kv_lens   as attn_decode_splitkv, with Lk_max = pages_per_seq * page_size
+ *   page_size         power of two, 16 <= page_size <= 65536
+ *   num_splits, workspace, ws_bytes  as attn_decode_splitkv with that Lk_max
+ *                     (attn_decode_workspace_size(B, Hq, Hkv, Lq,
+ *                      pages_per_seq * page_size, d, num_splits) bytes)
+ * Errors: as attn_decode_splitkv; INVALID_ARG also for a null or misaligned
+ * block_table or a bad page_size / pages_per_seq / num_pages.
+ */
+attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* block_table, void* o, float* lse,
+                                const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
+                                int page_size, int pages_per_seq, int num_pages, int d,
+                                float scale, int num_splits, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/*
  * attn_decode_splitkv_noalloc — attn_decode_splitkv for callers that cannot
  * allocate device memory.  (No counterpart on the pages: this is a library
  * convenience, not part of the method.)
@@ -183,7 +216,8 @@ attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* k_cache,
  * attn_get_device_error — synchronise `stream`, then read and clear the
  * device error word of the current device.  Returns ATTN_OK, ATTN_ERR_TIMEOUT
  * (a kernel abandoned a bounded wait), ATTN_ERR_INVALID_ARG (a kv_lens entry
- * was out of range) or ATTN_ERR_CUDA (the synchronisation itself failed).
+ * or a block_table page id was out of range) or ATTN_ERR_CUDA (the
+ * synchronisation itself failed).
  * `raw_bits` (nullable) receives the raw error bits.
  */
 attn_status_t attn_get_device_error(void* stream, int* raw_bits);

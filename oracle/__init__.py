@@ -63,6 +63,8 @@ def _load():
             lib.oracle_decode_partials.restype = i32
             lib.oracle_combine.argtypes = [P, P, i32, i64, i32, P, P]
             lib.oracle_combine.restype = i32
+            lib.oracle_paged_gather.argtypes = [P, P, i32, i32, i32, i32, i32, i32, P]
+            lib.oracle_paged_gather.restype = i32
             lib.oracle_max_threads.argtypes = []
             lib.oracle_max_threads.restype = i32
             _lib = lib
@@ -194,3 +196,19 @@ def combine(o_part, lse_part):
     if rc:
         raise ValueError("oracle_combine failed")
     return o, lse
+
+
+def paged_gather(pages, block_table):
+    """Logical cache [B, H, pages_per_seq * page_size, d] (bf16) from a page pool
+    [num_pages, H, page_size, d] (bf16) and a block table [B, pages_per_seq]."""
+    import torch
+    pb = _bf16_bits(pages)
+    num_pages, H, page_size, d = pb.shape
+    bt = _i32(block_table)
+    B, pps = bt.shape
+    out = np.zeros((B, H, pps * page_size, d), dtype=np.uint16)
+    rc = _load().oracle_paged_gather(_ptr(pb), _ptr(bt), B, H, page_size, pps, num_pages, d,
+                                     _ptr(out))
+    if rc:
+        raise ValueError("oracle_paged_gather: page id out of range or bad shape")
+    return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)

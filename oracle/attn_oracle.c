@@ -348,6 +348,35 @@ int oracle_combine(const double* o_part, const double* lse_part, int nsplit, int
   return 0;
 }
 
+/*
+ * Paged KV cache ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", section 1:
+ * PagedAttention maps logical to physical pages; section 4, experiment 1 runs
+ * the decode with a paged block_table): logical key j of sequence b lives in
+ * page block_table[b][j / page_size] at row j % page_size.  This writes the
+ * logical cache out contiguously so the plain attention above can run on it.
+ *   pages: [num_pages, H, page_size, d] (bf16 bits), out: [B, H, pages_per_seq*page_size, d].
+ * Returns -1 if a page id is out of range.
+ */
+int oracle_paged_gather(const uint16_t* pages, const int32_t* block_table, int B, int H,
+                        int page_size, int pages_per_seq, int num_pages, int d, uint16_t* out) {
+  if (B < 0 || H < 1 || page_size < 1 || pages_per_seq < 1 || num_pages < 1 || d < 1) return -1;
+  const int64_t L = (int64_t)pages_per_seq * page_size;
+  for (int b = 0; b < B; ++b) {
+    for (int i = 0; i < pages_per_seq; ++i) {
+      const int page = block_table[(int64_t)b * pages_per_seq + i];
+      if (page < 0 || page >= num_pages) return -1;
+      for (int h = 0; h < H; ++h) {
+        for (int r = 0; r < page_size; ++r) {
+          const uint16_t* src = pages + (((int64_t)page * H + h) * page_size + r) * d;
+          uint16_t* dst = out + (((int64_t)b * H + h) * L + (int64_t)i * page_size + r) * d;
+          for (int c = 0; c < d; ++c) dst[c] = src[c];
+        }
+      }
+    }
+  }
+  return 0;
+}
+
 int oracle_max_threads(void) {
 #ifdef _OPENMP
   return omp_get_max_threads();

@@ -26,8 +26,8 @@ __all__ = [
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
     "attn_fwd", "attn_decode_splitkv", "attn_decode_num_splits",
-    "attn_decode_workspace_size", "attn_decode_splitkv_noalloc", "attn_get_device_error",
-    "attn_selftest_wait_timeout", "attn_status_string",
+    "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
+    "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
     "EXPORTED_SYMBOLS",
 ]
 
@@ -45,8 +45,8 @@ _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 
 EXPORTED_SYMBOLS = (
     "attn_fwd", "attn_decode_num_splits", "attn_decode_workspace_size",
-    "attn_decode_splitkv", "attn_decode_splitkv_noalloc", "attn_get_device_error",
-    "attn_selftest_wait_timeout", "attn_status_string",
+    "attn_decode_splitkv", "attn_decode_paged", "attn_decode_splitkv_noalloc",
+    "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
 )
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,9 @@ def load_library():
         lib.attn_decode_splitkv.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32,
                                             i32, P, sz, P]
         lib.attn_decode_splitkv.restype = i32
+        lib.attn_decode_paged.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                          i32, f32, i32, P, sz, P]
+        lib.attn_decode_paged.restype = i32
         lib.attn_decode_splitkv_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32,
                                                     i32, f32, i32, P]
         lib.attn_decode_splitkv_noalloc.restype = i32
@@ -197,6 +200,40 @@ def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, *, scale=None, num_splits=
         workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_decode_splitkv")
+    return o, lse
+
+
+def attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, *, scale=None, num_splits=0,
+                      workspace=None, o=None, lse=None, stream=None):
+    """Split-KV decode over a paged cache (see ``attn_decode_paged`` in include/attn.h).
+
+    q: [B, Hq, Lq, d]; k_pages/v_pages: [num_pages, Hkv, page_size, d] bf16;
+    block_table: int32 [B, pages_per_seq]; kv_lens: int32 [B] (device).
+    """
+    for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
+        _check_bf16(name, t)
+    for name, t in (("block_table", block_table), ("kv_lens", kv_lens)):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+    B, Hq, Lq, d = q.shape
+    num_pages, Hkv, page_size, _ = k_pages.shape
+    pages_per_seq = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    need = attn_decode_workspace_size(B, Hq, Hkv, Lq, pages_per_seq * page_size, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    st = load_library().attn_decode_paged(
+        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(o), _ptr(lse),
+        _ptr(kv_lens), B, Hq, Hkv, Lq, page_size, pages_per_seq, num_pages, d, float(scale),
+        int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_decode_paged")
     return o, lse
 
 

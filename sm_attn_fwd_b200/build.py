@@ -36,9 +36,15 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def source_digest() -> str:
-    """Digest of the kernel sources and flags (identifies a profiled build)."""
-    return _digest()
+def source_digest(files=("attn_prefill.cu", "ptx.cuh", "attn_params.h")) -> str:
+    """Digest of one kernel's sources and the flags (identifies a profiled
+    build); by default the prefill kernel's."""
+    h = hashlib.sha256()
+    for name in files:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(NVCC_FLAGS).encode())
+    return h.hexdigest()[:16]
 
 
 def _digest() -> str:

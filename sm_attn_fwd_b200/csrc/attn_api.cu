@@ -50,14 +50,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// bf16 tensor map of rank 2 or 3 (innermost first), 64 x 128 boxes, 128-byte
-// swizzle; out-of-range rows read as zero.
-bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims) {
+// bf16 tensor map of rank 2 or 3 (innermost first), boxes of 64 columns by
+// box_rows rows, 128-byte swizzle; out-of-range rows read as zero.
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                 int box_rows = kBlockN) {
   auto fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[3];
   cuuint64_t gstride[2];
-  cuuint32_t box[3] = {64, (cuuint32_t)kBlockN, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estride[3] = {1, 1, 1};
   uint64_t stride = 2;
   for (int i = 0; i < rank; ++i) {
@@ -219,10 +220,22 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk_max, in
   return ws_lse_offset(pl, nrows, d) + (size_t)pl.nsplit * (size_t)nrows * 4;
 }
 
-attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
-                                  void* o, float* lse, const int32_t* kv_lens, int B, int Hq,
-                                  int Hkv, int Lq, int Lk_max, int d, float scale, int num_splits,
-                                  void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+struct PagedKv {
+  const int32_t* block_table = nullptr;
+  int page_size = 0;
+  int pages_per_seq = 0;
+  int num_pages = 0;
+};
+
+// Shared body of the contiguous and paged split-KV decode.
+attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o,
+                          float* lse, const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
+                          int Lk_max, int d, float scale, int num_splits, void* workspace,
+                          size_t ws_bytes, void* stream, const PagedKv& pg) {
   if (!q || !k_cache || !v_cache || !o || !lse || !kv_lens) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
       !aligned(lse, 4) || !aligned(kv_lens, 4))
@@ -260,13 +273,25 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
   p.chunk = pl.chunk;
   p.nsplit = pl.nsplit;
   p.row_tiles = pl.row_tiles;
+  p.block_table = pg.block_table;
+  p.page_size = pg.page_size;
+  p.pages_per_seq = pg.pages_per_seq;
+  p.num_pages = pg.num_pages;
 
   CUtensorMap tq, tk, tv;
   const uint64_t dq[2] = {(uint64_t)d, (uint64_t)nrows};
-  const uint64_t dk[3] = {(uint64_t)d, (uint64_t)Lk_max, (uint64_t)B * Hkv};
-  if (!encode_bf16(&tq, q, 2, dq) || !encode_bf16(&tk, k_cache, 3, dk) ||
-      !encode_bf16(&tv, v_cache, 3, dk))
-    return ATTN_ERR_CUDA;
+  if (!encode_bf16(&tq, q, 2, dq)) return ATTN_ERR_CUDA;
+  if (pg.block_table) {
+    const uint64_t dk[3] = {(uint64_t)d, (uint64_t)pg.page_size,
+                            (uint64_t)pg.num_pages * (uint64_t)Hkv};
+    const int rows = pg.page_size < kBlockN ? pg.page_size : kBlockN;
+    if (!encode_bf16(&tk, k_cache, 3, dk, rows) || !encode_bf16(&tv, v_cache, 3, dk, rows))
+      return ATTN_ERR_CUDA;
+  } else {
+    const uint64_t dk[3] = {(uint64_t)d, (uint64_t)Lk_max, (uint64_t)B * Hkv};
+    if (!encode_bf16(&tk, k_cache, 3, dk) || !encode_bf16(&tv, v_cache, 3, dk))
+      return ATTN_ERR_CUDA;
+  }
 
   dim3 grid((unsigned)pl.nsplit, (unsigned)(B * Hkv * pl.row_tiles), 1);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -275,6 +300,40 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   e = d == 64 ? attn::launch_combine<64>(p, st) : attn::launch_combine<128>(p, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                                  void* o, float* lse, const int32_t* kv_lens, int B, int Hq,
+                                  int Hkv, int Lq, int Lk_max, int d, float scale, int num_splits,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  return decode_impl(q, k_cache, v_cache, o, lse, kv_lens, B, Hq, Hkv, Lq, Lk_max, d, scale,
+                     num_splits, workspace, ws_bytes, stream, PagedKv{});
+}
+
+attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* block_table, void* o, float* lse,
+                                const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
+                                int page_size, int pages_per_seq, int num_pages, int d,
+                                float scale, int num_splits, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  if (!block_table || !aligned(block_table, 4)) return ATTN_ERR_INVALID_ARG;
+  if (page_size < 16 || page_size > (1 << 16) || (page_size & (page_size - 1)) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (pages_per_seq < 1 || num_pages < 1 || Hkv < 1) return ATTN_ERR_INVALID_ARG;
+  const long long lk = (long long)pages_per_seq * page_size;
+  if (lk > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)num_pages * Hkv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  PagedKv pg;
+  pg.block_table = block_table;
+  pg.page_size = page_size;
+  pg.pages_per_seq = pages_per_seq;
+  pg.num_pages = num_pages;
+  return decode_impl(q, k_pages, v_pages, o, lse, kv_lens, B, Hq, Hkv, Lq, (int)lk, d, scale,
+                     num_splits, workspace, ws_bytes, stream, pg);
 }
 
 attn_status_t attn_get_device_error(void* stream, int* raw_bits) {
@@ -293,7 +352,7 @@ attn_status_t attn_get_device_error(void* stream, int* raw_bits) {
   if (bits & (attn::kDevErrTimeoutProducer | attn::kDevErrTimeoutMma |
               attn::kDevErrTimeoutSoftmax | attn::kDevErrTimeoutSelftest))
     return ATTN_ERR_TIMEOUT;
-  if (bits & attn::kDevErrBadKvLen) return ATTN_ERR_INVALID_ARG;
+  if (bits & (attn::kDevErrBadKvLen | attn::kDevErrBadPage)) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
 

@@ -307,15 +307,55 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
-    if (lane == 0 && n_tiles > 0) {
+    // The whole warp runs this loop; lane 0 owns the barrier bookkeeping and the
+    // lanes share out the TMA boxes of a tile (many boxes for small pages).
+    if (n_tiles > 0) {
       constexpr uint32_t kTx = C::kTileBytes;
-      ptx::mbar_arrive_expect_tx(q_full, kTx);
-      for (int a = 0; a < C::kAtoms; ++a) {
-        if constexpr (kDecode)
-          ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y);
-        else
-          ptx::tma_load_3d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y, q_coord_z);
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(q_full, kTx);
+        for (int a = 0; a < C::kAtoms; ++a) {
+          if constexpr (kDecode)
+            ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y);
+          else
+            ptx::tma_load_3d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y,
+                             q_coord_z);
+        }
       }
+      // One 128-key K or V tile into shared memory.  Contiguous cache: one box
+      // per 64-column atom.  Paged cache ([num_pages, Hkv, page_size, d] through
+      // the block table): pages of 128 keys or more give one box per atom at
+      // the key's offset inside its page; smaller pages give one box per page
+      // slice, each landing on a whole number of 8-row swizzle atoms, so the
+      // assembled tile is laid out exactly like a single box.  Keys past the
+      // block table read as zeros (out-of-range coordinate), as do pages whose
+      // id is out of range (which also flags the device error word).
+      auto page_z = [&](int key) -> int {
+        const int idx = key / p.page_size;
+        if (idx >= p.pages_per_seq) return -1;
+        const int page = __ldg(p.block_table + (long long)b * p.pages_per_seq + idx);
+        if (page < 0 || page >= p.num_pages) {
+          atomicOr(&g_device_error, kDevErrBadPage);
+          return -1;
+        }
+        return page * p.Hkv + hkv;
+      };
+      auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int k0) {
+        if (p.block_table == nullptr) {
+          if (lane < C::kAtoms)
+            ptx::tma_load_3d(dst + lane * C::kAtomBytes, tm, bar, lane * 64, k0, kv_z);
+        } else if (p.page_size >= kBlockN) {
+          if (lane < C::kAtoms)
+            ptx::tma_load_3d(dst + lane * C::kAtomBytes, tm, bar, lane * 64, k0 % p.page_size,
+                             page_z(k0));
+        } else {
+          const int n_items = (kBlockN / p.page_size) * C::kAtoms;
+          for (int item = lane; item < n_items; item += 32) {
+            const int sub = item / C::kAtoms, a = item % C::kAtoms;
+            ptx::tma_load_3d(dst + a * C::kAtomBytes + sub * p.page_size * 128, tm, bar, a * 64,
+                             0, page_z(k0 + sub * p.page_size));
+          }
+        }
+      };
       int j = 0;
       bool ok = true;
       for (int t = t_lo; t <= t_hi && ok; ++t) {
@@ -325,34 +365,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int k0 = t * kBlockN;
         ok = ptx::mbar_wait(&k_empty[s], ph ^ 1u, abort_flag, &g_device_error,
                             kDevErrTimeoutProducer);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        ptx::mbar_arrive_expect_tx(&k_full[s], kTx);
-        for (int a = 0; a < C::kAtoms; ++a)
-          ptx::tma_load_3d(sK + s * C::kTileBytes + a * C::kAtomBytes, &tm_k, &k_full[s], a * 64,
-                           k0, kv_z);
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&k_full[s], kTx);
+        __syncwarp();
+        load_kv(sK + s * C::kTileBytes, &tm_k, &k_full[s], k0);
         ok = ptx::mbar_wait(&v_empty[s], ph ^ 1u, abort_flag, &g_device_error,
                             kDevErrTimeoutProducer);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) {
           ++j;  // the K load of this tile is in flight; drain it below
           break;
         }
-        ptx::mbar_arrive_expect_tx(&v_full[s], kTx);
-        for (int a = 0; a < C::kAtoms; ++a)
-          ptx::tma_load_3d(sV + s * C::kTileBytes + a * C::kAtomBytes, &tm_v, &v_full[s], a * 64,
-                           k0, kv_z);
+        if (lane == 0) ptx::mbar_arrive_expect_tx(&v_full[s], kTx);
+        __syncwarp();
+        load_kv(sV + s * C::kTileBytes, &tm_v, &v_full[s], k0);
         ++j;
       }
       // Drain: every TMA write into shared memory must land before the CTA exits.
       // In a normal run these phases have completed already.
-      int dummy_abort = 0;
-      ptx::mbar_wait(q_full, 0, &dummy_abort, nullptr, 0);
-      for (int jj = max(0, j - C::kStages); jj < j; ++jj) {
-        const int s = jj % C::kStages;
-        const uint32_t ph = (uint32_t)(jj / C::kStages) & 1u;
-        dummy_abort = 0;
-        ptx::mbar_wait(&k_full[s], ph, &dummy_abort, nullptr, 0);
-        dummy_abort = 0;
-        ptx::mbar_wait(&v_full[s], ph, &dummy_abort, nullptr, 0);
+      if (lane == 0) {
+        int dummy_abort = 0;
+        ptx::mbar_wait(q_full, 0, &dummy_abort, nullptr, 0);
+        for (int jj = max(0, j - C::kStages); jj < j; ++jj) {
+          const int s = jj % C::kStages;
+          const uint32_t ph = (uint32_t)(jj / C::kStages) & 1u;
+          dummy_abort = 0;
+          ptx::mbar_wait(&k_full[s], ph, &dummy_abort, nullptr, 0);
+          dummy_abort = 0;
+          ptx::mbar_wait(&v_full[s], ph, &dummy_abort, nullptr, 0);
+        }
       }
     }
   } else if (warp == 1) {

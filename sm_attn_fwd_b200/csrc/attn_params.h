@@ -19,6 +19,7 @@ enum DeviceError : int {
   kDevErrTimeoutSoftmax = 1 << 2,
   kDevErrBadKvLen = 1 << 3,
   kDevErrTimeoutSelftest = 1 << 4,
+  kDevErrBadPage = 1 << 5,
 };
 
 struct FwdParams {
@@ -43,6 +44,11 @@ struct FwdParams {
   int q_tiles;       // prefill: ceil(Lq / 128)
   int n_units;       // prefill: work units (pairs of query tiles x B*Hq)
   int* err;          // device error word
+  // paged KV cache (decode): K/V pages [num_pages, Hkv, page_size, d]
+  const int32_t* block_table;  // [B, pages_per_seq] page ids, or null (contiguous cache)
+  int page_size;               // keys per page (power of two, >= 16)
+  int pages_per_seq;           // row length of block_table; Lk = pages_per_seq * page_size
+  int num_pages;               // pages in the pool
 };
 
 }  // namespace attn

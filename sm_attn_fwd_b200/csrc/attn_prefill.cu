@@ -692,17 +692,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = r_row < w.rows[x];
       int row_lo = 0, row_hi = -1;  // visible key range, clamped to [0, Lk-1]
       int row_doc = 0;
-      const int32_t* doc_b = nullptr;
+      // document ids of this batch row (warp-uniform: every lane takes part in
+      // the ballots below, rows past Lq included)
+      const int32_t* doc_b = p.doc_ids ? p.doc_ids + (long long)w.b * p.Lk : nullptr;
       if (row_ok) {
         const long long pos = w.pos0[x] + r_row;
         long long lo, hi;
         key_bounds(p, pos, lo, hi);
         row_lo = (int)max(0LL, min(lo, (long long)p.Lk));
         row_hi = (int)max(-1LL, min(hi, (long long)p.Lk - 1));
-        if (p.doc_ids != nullptr) {
-          doc_b = p.doc_ids + (long long)w.b * p.Lk;
-          row_doc = __ldg(doc_b + pos);
-        }
+        if (doc_b != nullptr) row_doc = __ldg(doc_b + pos);
       }
       const int t_lo = s->t_lo, t_hi = s->t_hi;
       const int n_mine = s->n[x];
@@ -756,28 +755,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hi_rel = max(-1, min(127, row_hi - k0));
           uint32_t dm0 = ~0u, dm1 = ~0u, dm2 = ~0u, dm3 = ~0u;
           if (doc_b != nullptr) {
-            const int32_t* dk = doc_b + k0;
+            // lane i holds the document of keys k0 + 32g + i (g = 0..3); for each
+            // distinct row document in the warp one ballot per word gives every
+            // row with that document its visibility bits.  Keys past Lk are
+            // outside [lo_rel, hi_rel] whatever their bit says.
             const int kmax = min(128, p.Lk - k0);
-#pragma unroll 1
-            for (int g = 0; g < 4; ++g) {
-              uint32_t bits = 0;
+            int kd[4];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int kk = g * 32 + i;
-                const int dv = (kk < kmax) ? __ldg(dk + kk) : ~row_doc;
-                bits |= (dv == row_doc ? 1u : 0u) << i;
+            for (int g = 0; g < 4; ++g)
+              kd[g] = (32 * g + lane < kmax) ? __ldg(doc_b + k0 + 32 * g + lane) : 0;
+            uint32_t todo = 0xffffffffu;
+            while (todo != 0u) {  // at most 32 rounds: each clears its leader's bit
+              const int dv = __shfl_sync(0xffffffffu, row_doc, __ffs(todo) - 1);
+              const uint32_t same = __ballot_sync(0xffffffffu, row_doc == dv);
+              const uint32_t w0 = __ballot_sync(0xffffffffu, kd[0] == dv);
+              const uint32_t w1 = __ballot_sync(0xffffffffu, kd[1] == dv);
+              const uint32_t w2 = __ballot_sync(0xffffffffu, kd[2] == dv);
+              const uint32_t w3 = __ballot_sync(0xffffffffu, kd[3] == dv);
+              if ((same >> lane) & 1u) {
+                dm0 = w0;
+                dm1 = w1;
+                dm2 = w2;
+                dm3 = w3;
               }
-              if (g == 0) dm0 = bits;
-              else if (g == 1) dm1 = bits;
-              else if (g == 2) dm2 = bits;
-              else dm3 = bits;
+              todo &= ~same;
             }
+          }
+          // fold the key range into the four words: word g holds keys 32g..32g+31
+          {
+            auto range_bits = [&](int g) -> uint32_t {
+              const int a = lo_rel - 32 * g, b = hi_rel - 32 * g;
+              if (b < 0 || a > 31 || a > b) return 0u;
+              return (~0u << max(a, 0)) & (~0u >> (31 - min(b, 31)));
+            };
+            dm0 &= range_bits(0);
+            dm1 &= range_bits(1);
+            dm2 &= range_bits(2);
+            dm3 &= range_bits(3);
           }
 #pragma unroll
           for (int i = 0; i < 128; ++i) {
             const uint32_t word = i < 32 ? dm0 : (i < 64 ? dm1 : (i < 96 ? dm2 : dm3));
-            const bool vis = (i >= lo_rel) && (i <= hi_rel) && ((word >> (i & 31)) & 1u);
-            sv[i] = vis ? sv[i] : -INFINITY;
+            sv[i] = ((word >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
           }
         }
         // row max: eight independent chains of three-input max, then a tree
@@ -806,21 +825,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         float sum8[8];  // four packed (even, odd) partial sums
 #pragma unroll
         for (int j = 0; j < 8; ++j) sum8[j] = 0.0f;
+        // The exponentials of pair i are issued kAhead pairs before their sum
+        // and bf16 packing, so the MUFU results are ready when those read them
+        // and one warp keeps the unit fed (measured: 4 pairs ahead is best).
         auto emit_p = [&](auto fma_share) {
           constexpr bool kShare = decltype(fma_share)::value;
+          constexpr int kAhead = 4;
+          float e0[kAhead], e1[kAhead];
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int i0 = 2 * i, i1 = i0 + 1;
-            float a0, a1;
-            ptx::fma2_bc(a0, a1, sv[i0], sv[i1], c, -m_use);  // s * c - m, two at once
-            const float p0 = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
-            const float p1 = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
-            ptx::add2_acc(sum8[(i & 3) * 2], sum8[(i & 3) * 2 + 1], p0, p1);
-            const uint32_t packed = ptx::pack_bf16x2(p0, p1);
-            if (i < 16) pk0[i] = packed;
-            else if (i < 32) pk1[i - 16] = packed;
-            else if (i < 48) pk2[i - 32] = packed;
-            else pk3[i - 48] = packed;
+          for (int i = 0; i < 64 + kAhead; ++i) {
+            // slot i % kAhead: first consume pair i - kAhead, then refill it with pair i
+            if (i >= kAhead) {
+              const int j = i - kAhead;
+              const float p0 = e0[j % kAhead], p1 = e1[j % kAhead];
+              ptx::add2_acc(sum8[(j & 3) * 2], sum8[(j & 3) * 2 + 1], p0, p1);
+              const uint32_t packed = ptx::pack_bf16x2(p0, p1);
+              if (j < 16) pk0[j] = packed;
+              else if (j < 32) pk1[j - 16] = packed;
+              else if (j < 48) pk2[j - 32] = packed;
+              else pk3[j - 48] = packed;
+            }
+            if (i < 64) {
+              const int i0 = 2 * i, i1 = i0 + 1;
+              float a0, a1;
+              ptx::fma2_bc(a0, a1, sv[i0], sv[i1], c, -m_use);  // s * c - m, two at once
+              e0[i % kAhead] = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
+              e1[i % kAhead] = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
+            }
           }
         };
         ok = ptx::mbar_wait_a(bar_my_turn, (uint32_t)turns & 1u, abort_flag, err,
@@ -828,10 +859,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         ++turns;
-        if (full)
-          emit_p(std::true_type{});  // FULL tiles may send exponentials to the FMA pipe
-        else
-          emit_p(std::false_type{});  // PARTIAL tiles keep exact zeros at masked keys
+        // One copy of the loop in the instruction stream: a second copy (for
+        // PARTIAL tiles) measured 10% slower through instruction-cache misses.
+        if constexpr (kExpFmaShare) {
+          if (full)
+            emit_p(std::true_type{});  // FULL tiles may send exponentials to the FMA pipe
+          else
+            emit_p(std::false_type{});  // PARTIAL tiles keep exact zeros at masked keys
+        } else {
+          emit_p(std::false_type{});
+        }
         ptx::mbar_arrive_a(bar_other_turn);
 #pragma unroll
         for (int j = 0; j < 4; ++j) sum8[j] += sum8[j + 4];
@@ -848,7 +885,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tc_fence_after();
         }
         if (jl > 0 && any_need) {
-#pragma unroll
+#pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t raw[32];
             ptx::tmem_ld32(t_row + o_col + cc * 32, raw);
@@ -884,7 +921,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv_l = have ? 1.0f / l : 0.0f;
       const float lse_row = have ? (m_ref + ptx::lg2(l)) * kLn2 : -INFINITY;
       const long long out_row = (long long)w.bh * p.Lq + w.q0[x] + r_row;
-#pragma unroll
+#pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t raw[32];
         if (have_o && ok) {

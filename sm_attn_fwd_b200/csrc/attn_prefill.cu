@@ -799,17 +799,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[i] = ((word >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
           }
         }
-        // row max: eight independent chains of three-input max, then a tree
-        float mx8[8];
+        // row max: sixteen independent chains of two-input max, then a tree
+        float mx16[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) mx8[j] = fmaxf(sv[j], sv[8 + j]);
+        for (int j = 0; j < 16; ++j) mx16[j] = fmaxf(sv[j], sv[16 + j]);
 #pragma unroll
-        for (int i = 16; i < 128; i += 16) {
+        for (int i = 32; i < 128; i += 16) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) mx8[j] = ptx::max3(mx8[j], sv[i + j], sv[i + 8 + j]);
+          for (int j = 0; j < 16; ++j) mx16[j] = fmaxf(mx16[j], sv[i + j]);
         }
-        const float mx = fmaxf(ptx::max3(mx8[0], mx8[1], mx8[2]),
-                               ptx::max3(mx8[3], ptx::max3(mx8[4], mx8[5], mx8[6]), mx8[7]));
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+          for (int j = 0; j < w; ++j) mx16[j] = fmaxf(mx16[j], mx16[j + w]);
+        }
+        const float mx = mx16[0];
         const float m_new = fmaxf(m_ref, mx * c);
         const bool need = m_new > m_ref + kRescaleThreshold;
         const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;

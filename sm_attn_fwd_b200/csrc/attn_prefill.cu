@@ -479,9 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int last = s->last[x];
         bool first = true;
         // P_x V of key tile tp (union index jp), then release its V stage
-        auto issue_pv = [&](int tp, int jp) -> bool {
+        auto issue_pv = [&](int jp, bool mine) -> bool {
           const int stp = jp % S;
-          const bool mine = !bit_get(s->empty[x], tp - t_lo);
           bool w_ok = ptx::mbar_wait_a(V_FULL(stp), (uint32_t)(jp / S) & 1u, abort_flag, err,
                                        kDevErrTimeoutMma);
           if (w_ok && mine && first && r > 0)
@@ -503,10 +502,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           return true;
         };
         int t_prev = -1, j_prev = 0;
+        bool mine_prev = false;
+        // the schedule's bits for 32 key tiles at a time, in registers
+        int w_idx = -1;
+        uint32_t w_e0 = 0u, w_e1 = 0u;
         for (int t = t_lo; t <= t_hi && ok; ++t) {
-          if (!tile_used(s, t)) continue;
+          const int ti = t - t_lo;
+          if ((ti >> 5) != w_idx) {
+            w_idx = ti >> 5;
+            w_e0 = s->empty[0][w_idx];
+            w_e1 = s->empty[1][w_idx];
+          }
+          const uint32_t tbit = 1u << (ti & 31);
+          if (w_e0 & w_e1 & tbit) continue;  // no query tile of the unit uses key tile t
           const int st = jkv % S;
-          const bool mine = !bit_get(s->empty[x], t - t_lo);
+          const bool mine = ((x ? w_e1 : w_e0) & tbit) == 0u;
           // the softmax has loaded the previous S_x; K(t) has landed
           if (mine && ns > 0)
             ok = ptx::mbar_wait_a(BAR(kSFree + x), (uint32_t)(ns - 1) & 1u, abort_flag, err,
@@ -528,12 +538,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t == last) ptx::mma_commit_warp(BAR(kQEmpty + x));  // Q_x no longer read
           }
           ptx::mma_commit_warp(K_EMPTY(st));
-          if (t_prev >= 0) ok = issue_pv(t_prev, j_prev);
+          if (t_prev >= 0) ok = issue_pv(j_prev, mine_prev);
           t_prev = t;
           j_prev = jkv;
+          mine_prev = mine;
           ++jkv;
         }
-        if (ok && t_prev >= 0) ok = issue_pv(t_prev, j_prev);
+        if (ok && t_prev >= 0) ok = issue_pv(j_prev, mine_prev);
         if (last < 0) ptx::mma_commit_warp(BAR(kQEmpty + x));  // no key tile: Q_x unused
         if (lane == 0) ptx::mbar_arrive_a(BAR(kSchedEmpty + (r & 1)));
       }
@@ -708,9 +719,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       float m_ref = -INFINITY;
       float l = 0.0f;
       int jl = 0;
+      // the schedule's bits for 32 key tiles at a time, in registers
+      int w_idx = -1;
+      uint32_t w_e0 = 0u, w_e1 = 0u, w_full = 0u;
       for (int t = t_lo; t <= t_hi && ok; ++t) {
-        if (!tile_used(s, t)) continue;
-        if (bit_get(s->empty[x], t - t_lo)) {
+        const int ti = t - t_lo;
+        if ((ti >> 5) != w_idx) {
+          w_idx = ti >> 5;
+          w_e0 = s->empty[0][w_idx];
+          w_e1 = s->empty[1][w_idx];
+          w_full = s->full[x][w_idx];
+        }
+        const uint32_t tbit = 1u << (ti & 31);
+        if (w_e0 & w_e1 & tbit) continue;  // no query tile of the unit uses key tile t
+        if ((x ? w_e1 : w_e0) & tbit) {
           // no key tile of ours here: pass the turn on
           ok = ptx::mbar_wait_a(bar_my_turn, (uint32_t)turns & 1u, abort_flag, err,
                                 kDevErrTimeoutSoftmax);
@@ -719,7 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::mbar_arrive_a(bar_other_turn);
           continue;
         }
-        const bool full = bit_get(s->full[x], t - t_lo);
+        const bool full = (w_full & tbit) != 0u;
         const int k0 = t * 128;
         ok = ptx::mbar_wait_a(bar_s_full, (uint32_t)ns & 1u, abort_flag, err,
                               kDevErrTimeoutSoftmax);

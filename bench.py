@@ -420,6 +420,8 @@ def main():
                     help="with --only: multiply the batch (larger-than-L2 profiling case)")
     ap.add_argument("--batch", type=int, default=None,
                     help="with --only: set the batch size B (smaller profiling case)")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="with --only on a prefill workload: Lq = Lk = this length (profiling)")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: total CPU seconds across all steps")
@@ -445,6 +447,8 @@ def main():
         cfg = CONFIGS[args.only]
         if args.batch is not None:
             cfg = cfg.with_(B=args.batch, name=f"{cfg.name}_B{args.batch}")
+        if args.seq_len is not None and not cfg.decode:
+            cfg = cfg.with_(Lq=args.seq_len, Lk=args.seq_len, name=f"{cfg.name}_L{args.seq_len}")
         if cfg.decode:
             _, ms, nbytes, plan = run_decode(cfg, timer, args.steps, args.warmup, stream)
             print(json.dumps({"workload": cfg.name, "ms": ms, "GB/s": nbytes / (statistics.median(ms) * 1e6)}))

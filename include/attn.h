@@ -93,6 +93,41 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        void* stream);
 
 /*
+ * attn_fwd_varlen — prefill attention forward over packed sequences.
+ *
+ * The B sequences are packed one after another along the token axis with no
+ * padding ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", section 1: a
+ * document mask at the packing level; ragged lengths without padding).
+ * Sequence b owns query tokens [cu_seqlens_q[b], cu_seqlens_q[b+1]) and key
+ * tokens [cu_seqlens_k[b], cu_seqlens_k[b+1]); with Lq_b and Lk_b its lengths,
+ * its rows follow attn_fwd above with Lq = Lq_b, Lk = Lk_b (bottom-right
+ * alignment, the same mask kinds and window) and no document ids: a token
+ * never sees another sequence's keys.
+ *
+ * Arguments
+ *   q        [total_q, Hq, d] bf16, read (token-major, heads interleaved)
+ *   k, v     [total_k, Hkv, d] bf16, read
+ *   o        [total_q, Hq, d] bf16, written (rows of every sequence)
+ *   lse      [Hq, total_q] fp32, written
+ *   cu_seqlens_q, cu_seqlens_k  [B + 1] int32 in device memory, non-decreasing,
+ *            starting at 0 and ending at total_q / total_k
+ *   max_seqlen_q >= every Lq_b (sizes the grid); every Lk_b <= 524288
+ *   B, Hq, Hkv, total_q, total_k >= 1; d, scale, mask_kind, window_l,
+ *   window_r, draft_block as for attn_fwd
+ *   stream   cudaStream_t
+ * Errors: INVALID_ARG / UNSUPPORTED before any launch; CUDA on launch failure.
+ * cu_seqlens live in device memory, so the kernel checks them: a sequence whose
+ * bounds are out of order or out of range, or longer than max_seqlen_q, is
+ * skipped and flagged in the device error word (attn_get_device_error then
+ * returns ATTN_ERR_INVALID_ARG).
+ */
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                              int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
+                              float scale, int mask_kind, int window_l, int window_r,
+                              int draft_block, void* stream);
+
+/*
  * attn_decode_num_splits — how many KV splits attn_decode_splitkv uses.
  *
  * The keys [0, Lk_max) are cut into nsplit chunks of `chunk` keys each, a

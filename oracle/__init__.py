@@ -212,3 +212,44 @@ def paged_gather(pages, block_table):
     if rc:
         raise ValueError("oracle_paged_gather: page id out of range or bad shape")
     return torch.from_numpy(out.view(np.int16)).view(torch.bfloat16)
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale=None, mask="none",
+                    window=(-1, -1), draft_block=1):
+    """Packed sequences: the plain definition applied to each sequence on its own.
+
+    q: [total_q, Hq, d] bf16, k, v: [total_k, Hkv, d] bf16 (token-major);
+    sequence b owns query tokens cu_seqlens_q[b]:cu_seqlens_q[b+1] and key tokens
+    cu_seqlens_k[b]:cu_seqlens_k[b+1] ("FlexAttention 是什么，以及 DFlash2 之谜的完整
+    侦破", section 1: a document mask at the packing level, ragged lengths without
+    padding).  Each sequence is attention with Lq = Lq_b, Lk = Lk_b as in
+    ``attn_fwd``; a row with no key gets O = 0, LSE = -inf.  Returns (O, LSE) as
+    float64 numpy arrays shaped [total_q, Hq, d] and [Hq, total_q].
+    """
+    import torch
+    cq = np.asarray(_i32(cu_seqlens_q), dtype=np.int64)
+    ck = np.asarray(_i32(cu_seqlens_k), dtype=np.int64)
+    if cq.shape != ck.shape or cq.ndim != 1 or cq.size < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 entries")
+    total_q, Hq, d = q.shape
+    total_k, Hkv, _ = k.shape
+    if cq[0] != 0 or ck[0] != 0 or cq[-1] != total_q or ck[-1] != total_k:
+        raise ValueError("cu_seqlens must start at 0 and end at the token counts")
+    if np.any(np.diff(cq) < 0) or np.any(np.diff(ck) < 0):
+        raise ValueError("cu_seqlens must be non-decreasing")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    o = np.zeros((total_q, Hq, d), dtype=np.float64)
+    lse = np.full((Hq, total_q), -np.inf, dtype=np.float64)
+    for b in range(cq.size - 1):
+        q0, q1, k0, k1 = int(cq[b]), int(cq[b + 1]), int(ck[b]), int(ck[b + 1])
+        if q1 == q0 or k1 == k0:
+            continue  # no rows, or rows with no key (O = 0, LSE = -inf)
+        qb = q[q0:q1].permute(1, 0, 2).unsqueeze(0).contiguous()
+        kb = k[k0:k1].permute(1, 0, 2).unsqueeze(0).contiguous()
+        vb = v[k0:k1].permute(1, 0, 2).unsqueeze(0).contiguous()
+        ob, lb = attn_fwd(qb, kb, vb, scale=scale, mask=mask, window=window,
+                          draft_block=draft_block)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[:, q0:q1] = lb[0]
+    return o, lse

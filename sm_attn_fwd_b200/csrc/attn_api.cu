@@ -352,7 +352,8 @@ attn_status_t attn_get_device_error(void* stream, int* raw_bits) {
   if (bits & (attn::kDevErrTimeoutProducer | attn::kDevErrTimeoutMma |
               attn::kDevErrTimeoutSoftmax | attn::kDevErrTimeoutSelftest))
     return ATTN_ERR_TIMEOUT;
-  if (bits & (attn::kDevErrBadKvLen | attn::kDevErrBadPage)) return ATTN_ERR_INVALID_ARG;
+  if (bits & (attn::kDevErrBadKvLen | attn::kDevErrBadPage | attn::kDevErrBadSeqlens))
+    return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
 }
 

@@ -20,6 +20,7 @@ enum DeviceError : int {
   kDevErrBadKvLen = 1 << 3,
   kDevErrTimeoutSelftest = 1 << 4,
   kDevErrBadPage = 1 << 5,
+  kDevErrBadSeqlens = 1 << 6,
 };
 
 struct FwdParams {
@@ -44,6 +45,10 @@ struct FwdParams {
   int q_tiles;       // prefill: ceil(Lq / 128)
   int n_units;       // prefill: work units (pairs of query tiles x B*Hq)
   int* err;          // device error word
+  // packed sequences (prefill): null for the [B, H, L, d] layout
+  const int32_t* cu_seqlens_q;  // [B + 1]
+  const int32_t* cu_seqlens_k;  // [B + 1]
+  int total_q, total_k;         // tokens in the packed Q and K/V tensors
   // paged KV cache (decode): K/V pages [num_pages, Hkv, page_size, d]
   const int32_t* block_table;  // [B, pages_per_seq] page ids, or null (contiguous cache)
   int page_size;               // keys per page (power of two, >= 16)

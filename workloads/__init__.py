@@ -153,3 +153,29 @@ def random_case(seed, B, Hq, Hkv, Lq, Lk, d, *, factor=1.0, device="cpu", doc_sp
         lo, hi = kv_len_range
         kv_lens = torch.randint(lo, hi + 1, (B,), generator=g, device=device).to(torch.int32)
     return q, k, v, doc_ids, kv_lens
+
+
+def packed_case(seed, lens_q, lens_k, Hq, Hkv, d, *, factor=1.0, device="cpu"):
+    """Packed (token-major) sequences: Q [total_q, Hq, d], K and V [total_k, Hkv, d],
+    bf16 from the same recipe (Q, K, V drawn in that order), and the int32
+    cu_seqlens [B + 1] of both sides."""
+    device = torch.device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    tq, tk = int(sum(lens_q)), int(sum(lens_k))
+    q = _randn_bf16((tq, Hq, d), g, device, factor)
+    k = _randn_bf16((tk, Hkv, d), g, device, factor)
+    v = _randn_bf16((tk, Hkv, d), g, device, factor)
+    cu_q = torch.tensor([0] + [int(x) for x in torch.tensor(lens_q).cumsum(0)], dtype=torch.int32,
+                        device=device)
+    cu_k = torch.tensor([0] + [int(x) for x in torch.tensor(lens_k).cumsum(0)], dtype=torch.int32,
+                        device=device)
+    return q, k, v, cu_q, cu_k
+
+
+def packed_lengths(seed, n, lo, hi):
+    """n sequence lengths drawn uniformly from [lo, hi] (the length mix of a
+    packed batch of documents)."""
+    g = torch.Generator()
+    g.manual_seed(seed)
+    return [int(x) for x in torch.randint(lo, hi + 1, (n,), generator=g)]

@@ -228,6 +228,29 @@ def run_prefill(cfg, timer, steps, warmup, stream, batch_mult=1):
     return c, inp, ms, algorithmic_flops(c, pairs)
 
 
+# Packed sequences: 16 documents with lengths drawn uniformly from [128, 4096]
+# (seed 5), self-attention, causal, H = 16, d = 64.
+VARLEN_NAME = "varlen_causal_16seqs_l128to4096_h16_d64"
+
+
+def run_varlen(timer, steps, warmup, stream, *, n=16, lo=128, hi=4096, H=16, d=64, seed=5):
+    import sm_attn_fwd_b200 as ab
+    from workloads import packed_case, packed_lengths
+    lens = packed_lengths(seed, n, lo, hi)
+    q, k, v, cu_q, cu_k = packed_case(seed, lens, lens, H, H, d, device="cuda")
+    torch.cuda.synchronize()
+    o = torch.empty_like(q)
+    lse = torch.empty(H, q.shape[0], dtype=torch.float32, device="cuda")
+    fn = lambda: ab.attn_fwd_varlen(q, k, v, cu_q, cu_k, max(lens), mask="causal", o=o,  # noqa: E731
+                                    lse=lse, stream=stream)
+    ms = timer.time(fn, steps, warmup)
+    st, bits = ab.attn_get_device_error(stream)
+    if st != ab.ATTN_OK:
+        raise RuntimeError(f"device error after {VARLEN_NAME}: {st} {bits}")
+    pairs = sum(L * (L + 1) // 2 for L in lens)
+    return ms, 4.0 * d * pairs * H, lens
+
+
 def run_decode(cfg, timer, steps, warmup, stream):
     import sm_attn_fwd_b200 as ab
     inp = make_inputs(cfg, device="cuda")
@@ -472,6 +495,12 @@ def main():
                 workloads[c2.name] = {"ms_median": med, "ms_min": min(ms2), "TFLOP/s": tf,
                                       "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
                                       "algorithmic_flop": fl2}
+            ms5, fl5, lens5 = run_varlen(timer, max(5, args.steps // 10), 3, stream)
+            med = statistics.median(ms5)
+            tf = fl5 / (med * 1e9)
+            workloads[VARLEN_NAME] = {"ms_median": med, "ms_min": min(ms5), "TFLOP/s": tf,
+                                      "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                                      "algorithmic_flop": fl5, "tokens": sum(lens5)}
             for dc in (DECODE_LQ1, DECODE_LQ16):
                 _, ms3, nb, plan = run_decode(dc, timer, max(5, args.steps // 10), 3, stream)
                 med = statistics.median(ms3)

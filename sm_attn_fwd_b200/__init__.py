@@ -25,7 +25,7 @@ __all__ = [
     "AttnError", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
-    "attn_fwd", "attn_decode_splitkv", "attn_decode_num_splits",
+    "attn_fwd", "attn_fwd_varlen", "attn_decode_splitkv", "attn_decode_num_splits",
     "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
     "EXPORTED_SYMBOLS",
@@ -44,7 +44,7 @@ MASK_DRAFT_BLOCK = 2
 _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 
 EXPORTED_SYMBOLS = (
-    "attn_fwd", "attn_decode_num_splits", "attn_decode_workspace_size",
+    "attn_fwd", "attn_fwd_varlen", "attn_decode_num_splits", "attn_decode_workspace_size",
     "attn_decode_splitkv", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
 )
@@ -79,6 +79,9 @@ def load_library():
         lib.attn_fwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, i32,
                                  i32, P, P]
         lib.attn_fwd.restype = i32
+        lib.attn_fwd_varlen.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32,
+                                        i32, i32, i32, i32, P]
+        lib.attn_fwd_varlen.restype = i32
         lib.attn_decode_num_splits.argtypes = [i32] * 7 + [ctypes.POINTER(ctypes.c_int)]
         lib.attn_decode_num_splits.restype = i32
         lib.attn_decode_workspace_size.argtypes = [i32] * 7
@@ -116,13 +119,13 @@ def _stream_handle(stream, device):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _check_bf16(name, t):
+def _check_bf16(name, t, layout="[B, H, L, D]"):
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if t.dtype != torch.bfloat16:
         raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
-    if t.dim() != 4 or not t.is_contiguous():
-        raise ValueError(f"{name} must be a contiguous [B, H, L, D] tensor")
+    if t.dim() != layout.count(",") + 1 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {layout} tensor")
 
 
 def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
@@ -151,6 +154,41 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
                                  int(draft_block), _ptr(doc_ids), _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, *, scale=None,
+                    mask="none", window=(-1, -1), draft_block=1, o=None, lse=None, stream=None):
+    """Prefill forward over packed sequences (see ``attn_fwd_varlen`` in include/attn.h).
+
+    q: [total_q, Hq, d], k/v: [total_k, Hkv, d] bf16 CUDA tensors (token-major);
+    cu_seqlens_q/k: int32 CUDA tensors [B + 1].  Returns (o bf16 [total_q, Hq, d],
+    lse fp32 [Hq, total_q]).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_bf16(name, t, "[total, H, D]")
+    total_q, Hq, d = q.shape
+    total_k, Hkv, _ = k.shape
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.dim() != 1:
+            raise ValueError(f"{name} must be a contiguous int32 CUDA tensor [B + 1]")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both have B + 1 >= 2 entries")
+    B = cu_seqlens_q.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    mk = mask if isinstance(mask, int) else _MASKS[mask]
+    st = load_library().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                        _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, Hq, Hkv, total_q,
+                                        total_k, int(max_seqlen_q), d, float(scale), mk,
+                                        int(window[0]), int(window[1]), int(draft_block),
+                                        _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_varlen")
     return o, lse
 
 

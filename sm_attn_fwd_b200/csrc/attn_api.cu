@@ -73,6 +73,23 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
   return r == CUDA_SUCCESS;
 }
 
+// Token-major packed tensor [total, H, d]: dims {d, H, total}, one head per
+// box row group: box {64 columns, 1 head, 128 tokens}, the same shared-memory
+// image as a 128-row box of the [B, H, L, d] layout.
+bool encode_bf16_packed(CUtensorMap* map, const void* base, int d, int H, int total) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
+  cuuint64_t gstride[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kBlockN};
+  cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3u, const_cast<void*>(base), gdim,
+                  gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) {
@@ -195,6 +212,62 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   const uint64_t dq[3] = {(uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq};
   const uint64_t dk[3] = {(uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv};
   if (!encode_bf16(&tq, q, 3, dq) || !encode_bf16(&tk, k, 3, dk) || !encode_bf16(&tv, v, 3, dk))
+    return ATTN_ERR_CUDA;
+
+  const int grid = (int)(n_units < num_sms() ? n_units : num_sms());
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = d == 64 ? attn::launch_prefill<64>(tq, tk, tv, p, grid, st)
+                          : attn::launch_prefill<128>(tq, tk, tv, p, grid, st);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                              int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
+                              float scale, int mask_kind, int window_l, int window_r,
+                              int draft_block, void* stream) {
+  if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (total_q < 1 || total_k < 1 || max_seqlen_q < 1 || max_seqlen_q > total_q)
+    return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_DRAFT_BLOCK) return ATTN_ERR_INVALID_ARG;
+  if (window_l < -1 || window_r < -1) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_DRAFT_BLOCK && draft_block < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+
+  FwdParams p;
+  std::memset(&p, 0, sizeof p);
+  p.o = o;
+  p.lse = lse;
+  p.cu_seqlens_q = cu_seqlens_q;
+  p.cu_seqlens_k = cu_seqlens_k;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = max_seqlen_q;  // sizes the units; each sequence's lengths come from cu_seqlens
+  p.Lk = 0;
+  p.group = Hq / Hkv;
+  p.mask_kind = mask_kind;
+  p.window_l = window_l;
+  p.window_r = window_r;
+  p.draft_block = mask_kind == ATTN_MASK_DRAFT_BLOCK ? draft_block : 1;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.q_tiles = (int)ceil_div(max_seqlen_q, kBlockM);
+  const long long n_units = (long long)B * Hq * ((p.q_tiles + 1) / 2);
+  if (n_units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  p.n_units = (int)n_units;
+  p.err = error_word_for_current_device();
+  if (!p.err) return ATTN_ERR_CUDA;
+
+  CUtensorMap tq, tk, tv;
+  if (!encode_bf16_packed(&tq, q, d, Hq, total_q) || !encode_bf16_packed(&tk, k, d, Hkv, total_k) ||
+      !encode_bf16_packed(&tv, v, d, Hkv, total_k))
     return ATTN_ERR_CUDA;
 
   const int grid = (int)(n_units < num_sms() ? n_units : num_sms());

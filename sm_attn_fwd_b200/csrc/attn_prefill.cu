@@ -99,19 +99,22 @@ enum : int {
 
 struct Unit {
   int b, hq, hkv, bh;
-  int q0[2];        // first query row of tile A / B
+  int q0[2];        // first query row of tile A / B (within its sequence)
   int rows[2];      // valid rows of tile A / B (0 if the tile is past Lq)
   long long pos0[2];  // absolute position of row 0 of tile A / B
+  int Lk;           // keys of the sequence
+  int q_base, k_base;  // packed sequences: first token of the sequence in Q and in K/V
+  bool bad;         // packed sequences: out-of-range cu_seqlens (the unit is skipped)
 };
 
 __device__ __forceinline__ long long floor_div_ll(long long a, long long b) {
   return a >= 0 ? a / b : -((-a + b - 1) / b);
 }
 
-__device__ __forceinline__ void key_bounds(const FwdParams& p, long long pos, long long& lo,
-                                           long long& hi) {
+__device__ __forceinline__ void key_bounds(const FwdParams& p, int Lk, long long pos,
+                                           long long& lo, long long& hi) {
   lo = 0;
-  hi = (long long)p.Lk - 1;
+  hi = (long long)Lk - 1;
   if (p.mask_kind == kMaskCausal) {
     hi = min(hi, pos);
   } else if (p.mask_kind == kMaskDraftBlock) {
@@ -151,21 +154,42 @@ __device__ __forceinline__ bool bit_get(const uint32_t* bits, int i) {
   return (bits[i >> 5] >> (i & 31)) & 1u;
 }
 
-// The u-th unit (0 = heaviest): pairs of query tiles, last pair first.
+// The u-th unit (0 = heaviest): pairs of query tiles, last pair first.  With
+// packed sequences, unit u is the pair `u / (B*Hq)` places before the last
+// pair of its sequence (units past a short sequence's first pair are empty).
 __device__ __forceinline__ void decode_unit(const FwdParams& p, int u, Unit& w) {
   const int BH = p.B * p.Hq;
   const int n_pairs = (p.q_tiles + 1) / 2;
-  const int pair = n_pairs - 1 - u / BH;
   w.bh = u % BH;
   w.b = w.bh / p.Hq;
   w.hq = w.bh % p.Hq;
   w.hkv = w.hq / p.group;
+  int Lq = p.Lq, pair = n_pairs - 1 - u / BH;
+  w.Lk = p.Lk;
+  w.q_base = w.k_base = 0;
+  w.bad = false;
+  if (p.cu_seqlens_q != nullptr) {
+    const int cq0 = __ldg(p.cu_seqlens_q + w.b), cq1 = __ldg(p.cu_seqlens_q + w.b + 1);
+    const int ck0 = __ldg(p.cu_seqlens_k + w.b), ck1 = __ldg(p.cu_seqlens_k + w.b + 1);
+    Lq = cq1 - cq0;
+    const int pairs_b = ((Lq + 127) / 128 + 1) / 2;  // <= n_pairs when Lq <= p.Lq
+    w.bad = cq0 < 0 || cq1 < cq0 || cq1 > p.total_q || ck0 < 0 || ck1 < ck0 ||
+            ck1 > p.total_k || ck1 - ck0 > kMaxKvTiles * kBlockN || Lq > p.Lq;
+    pair = pairs_b - 1 - u / BH;
+    if (w.bad || pair < 0) {  // nothing to do: no rows in either tile
+      Lq = 0;
+      pair = 0;
+    }
+    w.Lk = w.bad ? 0 : ck1 - ck0;
+    w.q_base = w.bad ? 0 : cq0;
+    w.k_base = w.bad ? 0 : ck0;
+  }
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
     const int q0 = (2 * pair + x) * 128;
     w.q0[x] = q0;
-    w.rows[x] = max(0, min(128, p.Lq - q0));
-    w.pos0[x] = (long long)p.Lk - p.Lq + q0;
+    w.rows[x] = max(0, min(128, Lq - q0));
+    w.pos0[x] = (long long)w.Lk - Lq + q0;
   }
 }
 
@@ -187,8 +211,8 @@ __device__ void build_sched(const FwdParams& p, const Unit& w, Sched* s, int lan
     lo_first[x] = hi_last[x] = 0;
     hi_first[x] = lo_last[x] = -1;
     if (w.rows[x] > 0) {
-      key_bounds(p, w.pos0[x], lo_first[x], hi_first[x]);
-      key_bounds(p, w.pos0[x] + w.rows[x] - 1, lo_last[x], hi_last[x]);
+      key_bounds(p, w.Lk, w.pos0[x], lo_first[x], hi_first[x]);
+      key_bounds(p, w.Lk, w.pos0[x] + w.rows[x] - 1, lo_last[x], hi_last[x]);
       if (hi_last[x] >= lo_first[x] && hi_last[x] >= 0) {
         any[x] = true;
         t_lo = min(t_lo, (int)(lo_first[x] / 128));
@@ -228,7 +252,7 @@ __device__ void build_sched(const FwdParams& p, const Unit& w, Sched* s, int lan
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
       empty[x] = (i >= ntc) || !any[x] || k0 > hi_last[x] || k0 + 127 < lo_first[x];
-      full[x] = !empty[x] && (k0 + 128 <= p.Lk) && (lo_last[x] <= k0) &&
+      full[x] = !empty[x] && (k0 + 128 <= w.Lk) && (lo_last[x] <= k0) &&
                 (hi_first[x] >= k0 + 127);
     }
     if (doc_b) {
@@ -328,6 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
+  const bool packed = p.cu_seqlens_q != nullptr;  // token-major packed sequences
 
   if (threadIdx.x == 0) {
     ptx::prefetch_tmap(&tm_q);
@@ -382,6 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         rounds = r + 1;
         Unit w;
         decode_unit(p, u, w);
+        if (w.bad && lane == 0) atomicOr(err, kDevErrBadSeqlens);
         Sched* s = &scheds[r & 1];
         ok = ptx::mbar_wait_a(BAR(kSchedEmpty + (r & 1)), (((uint32_t)r >> 1) & 1u) ^ 1u,
                               abort_flag, err, kDevErrTimeoutProducer);
@@ -396,12 +422,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = ptx::mbar_wait_a(BAR(kQEmpty + x), ((uint32_t)r & 1u) ^ 1u, abort_flag, err,
                                   kDevErrTimeoutProducer);
             if (!ok) break;
+            if (w.rows[x] == 0) {  // tile past the sequence: nothing reads Q_x
+              ptx::mbar_arrive_a(BAR(kQFull + x));
+              continue;
+            }
             ptx::mbar_arrive_expect_tx_a(BAR(kQFull + x), kTx);
+            // [B, Hq, Lq, d]: (column, row, b*Hq + hq); packed: (column, hq, token)
+            const int qy = packed ? w.hq : w.q0[x];
+            const int qz = packed ? w.q_base + w.q0[x] : w.bh;
             for (int a = 0; a < C::kAtoms; ++a)
               ptx::tma_load_3d_a(sq + x * C::kTileBytes + a * C::kAtomBytes, &tm_q,
-                                 BAR(kQFull + x), a * 64, w.q0[x], w.bh);
+                                 BAR(kQFull + x), a * 64, qy, qz);
           }
-          const int kv_z = w.b * p.Hkv + w.hkv;
+          // [B, Hkv, Lk, d]: (column, key, b*Hkv + hkv); packed: (column, hkv, token)
+          const int kv_z = packed ? 0 : w.b * p.Hkv + w.hkv;
           const int t_hi = s->t_hi;
           for (int t = s->t_lo; t <= t_hi && ok; ++t) {
             if (!tile_used(s, t)) continue;
@@ -412,7 +446,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_arrive_expect_tx_a(K_FULL(st), kTx);
             for (int a = 0; a < C::kAtoms; ++a)
               ptx::tma_load_3d_a(sk + st * C::kTileBytes + a * C::kAtomBytes, &tm_k, K_FULL(st),
-                                 a * 64, t * 128, kv_z);
+                                 a * 64, packed ? w.hkv : t * 128,
+                                 packed ? w.k_base + t * 128 : kv_z);
             ok = ptx::mbar_wait_a(V_EMPTY(st), ph ^ 1u, abort_flag, err, kDevErrTimeoutProducer);
             if (!ok) {
               ++jkv;  // its K load is in flight: drain it below
@@ -421,7 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_arrive_expect_tx_a(V_FULL(st), kTx);
             for (int a = 0; a < C::kAtoms; ++a)
               ptx::tma_load_3d_a(sv_ + st * C::kTileBytes + a * C::kAtomBytes, &tm_v, V_FULL(st),
-                                 a * 64, t * 128, kv_z);
+                                 a * 64, packed ? w.hkv : t * 128,
+                                 packed ? w.k_base + t * 128 : kv_z);
             ++jkv;
           }
         }
@@ -709,9 +745,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (row_ok) {
         const long long pos = w.pos0[x] + r_row;
         long long lo, hi;
-        key_bounds(p, pos, lo, hi);
-        row_lo = (int)max(0LL, min(lo, (long long)p.Lk));
-        row_hi = (int)max(-1LL, min(hi, (long long)p.Lk - 1));
+        key_bounds(p, w.Lk, pos, lo, hi);
+        row_lo = (int)max(0LL, min(lo, (long long)w.Lk));
+        row_hi = (int)max(-1LL, min(hi, (long long)w.Lk - 1));
         if (doc_b != nullptr) row_doc = __ldg(doc_b + pos);
       }
       const int t_lo = s->t_lo, t_hi = s->t_hi;
@@ -946,7 +982,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool have = have_o && ok && l > 0.0f;
       const float inv_l = have ? 1.0f / l : 0.0f;
       const float lse_row = have ? (m_ref + ptx::lg2(l)) * kLn2 : -INFINITY;
-      const long long out_row = (long long)w.bh * p.Lq + w.q0[x] + r_row;
+      // [B, Hq, Lq, d] / [B, Hq, Lq]; packed: [total_q, Hq, d] / [Hq, total_q]
+      const long long tok = (long long)w.q_base + w.q0[x] + r_row;
+      const long long out_row = packed ? tok * p.Hq + w.hq : (long long)w.bh * p.Lq + w.q0[x] + r_row;
+      const long long lse_idx = packed ? (long long)w.hq * p.total_q + tok : out_row;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t raw[32];
@@ -974,7 +1013,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (row_ok) p.lse[out_row] = lse_row;
+      if (row_ok) p.lse[lse_idx] = lse_row;
       ptx::tc_fence_before();
       ptx::mbar_arrive_a(bar_o_free);
     }

@@ -112,3 +112,27 @@ def test_decode_rejects_on_host():
     no_ws = list(args)
     no_ws[14] = None
     assert lib.attn_decode_splitkv(*no_ws) == ab.ATTN_ERR_WORKSPACE
+
+
+def test_attn_fwd_varlen_rejects_on_host():
+    lib = ab.load_library()
+    #      q  k  v  o  lse cu_q cu_k B  Hq Hkv tq   tk   maxq d   scale mask wl  wr bd stream
+    args = [A, A, A, A, A, A, A, 3, 8, 2, 500, 600, 300, 128, 0.125, 1, -1, -1, 1, None]
+
+    def call(**over):
+        a = list(args)
+        for i, v in over.items():
+            a[int(i[1:])] = v
+        return lib.attn_fwd_varlen(*a)
+
+    assert call(a5=None) == ab.ATTN_ERR_INVALID_ARG        # no cu_seqlens_q
+    assert call(a6=ctypes.c_void_p(0x10002)) == ab.ATTN_ERR_INVALID_ARG  # cu_seqlens_k not int32-aligned
+    assert call(a0=M) == ab.ATTN_ERR_INVALID_ARG           # q not 16-byte aligned
+    assert call(a9=3) == ab.ATTN_ERR_INVALID_ARG           # Hq % Hkv != 0
+    assert call(a12=0) == ab.ATTN_ERR_INVALID_ARG          # max_seqlen_q < 1
+    assert call(a12=501) == ab.ATTN_ERR_INVALID_ARG        # max_seqlen_q > total_q
+    assert call(a10=0) == ab.ATTN_ERR_INVALID_ARG          # total_q < 1
+    assert call(a14=0.0) == ab.ATTN_ERR_INVALID_ARG        # scale
+    assert call(a15=2, a18=0) == ab.ATTN_ERR_INVALID_ARG   # draft block < 1
+    assert call(a16=-2) == ab.ATTN_ERR_INVALID_ARG         # window < -1
+    assert call(a13=96) == ab.ATTN_ERR_UNSUPPORTED         # d

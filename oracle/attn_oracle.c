@@ -160,10 +160,14 @@ int64_t oracle_count_pairs(int B, int Lq, int Lk, int mask_kind, int window_l, i
  */
 static double attend_row(const uint16_t* q_row, const uint16_t* k_head, const uint16_t* v_head,
                          int d, double scale, const mask_spec* m, int b, int i, int j_lo,
-                         int j_hi, double* s_buf, uint8_t* ok_buf, double* q_buf,
-                         double* o_row) {
+                         int j_hi, double alibi_slope, double* s_buf, uint8_t* ok_buf,
+                         double* q_buf, double* o_row) {
   for (int c = 0; c < d; ++c) q_buf[c] = bf16_bits_to_double(q_row[c]);
-  /* scores of the row: S_ij = scale * sum_c Q_ic K_jc */
+  /* scores of the row: S_ij = scale * sum_c Q_ic K_jc, then the score_mod
+     ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", section 1: score_mod(score,
+     b, h, q_idx, kv_idx), e.g. ALiBi): S_ij += slope_h * (j - p), p the row's
+     absolute position; slope 0 leaves the scores as they are */
+  const double p_abs = (double)(key_count(m, b) - m->Lq + i);
   int any = 0;
   for (int j = j_lo; j < j_hi; ++j) {
     ok_buf[j - j_lo] = (uint8_t)allowed(m, b, i, j);
@@ -171,7 +175,7 @@ static double attend_row(const uint16_t* q_row, const uint16_t* k_head, const ui
     const uint16_t* k_row = k_head + (int64_t)j * d;
     double acc = 0.0;
     for (int c = 0; c < d; ++c) acc += q_buf[c] * bf16_bits_to_double(k_row[c]);
-    s_buf[j - j_lo] = scale * acc;
+    s_buf[j - j_lo] = scale * acc + alibi_slope * ((double)j - p_abs);
     any = 1;
   }
   for (int c = 0; c < d; ++c) o_row[c] = 0.0;
@@ -205,11 +209,11 @@ static int check_shapes(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
  * (b * Hq + hq) * Lq + i; rows == NULL means every row in order.
  * o is [nrows, d], lse is [nrows].
  */
-int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+static int attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
                      int Hkv, int Lq, int Lk, int d, double scale, int mask_kind, int window_l,
                      int window_r, int draft_block, const int32_t* doc_ids,
-                     const int32_t* kv_lens, const int64_t* rows, int64_t nrows, double* o,
-                     double* lse, int nthreads) {
+                     const int32_t* kv_lens, const double* alibi_slopes, const int64_t* rows,
+                     int64_t nrows, double* o, double* lse, int nthreads) {
   if (check_shapes(B, Hq, Hkv, Lq, Lk, d)) return -1;
   mask_spec m = {B, Lq, Lk, mask_kind, window_l, window_r, draft_block, doc_ids, kv_lens};
   if (check_mask_spec(&m)) return -1;
@@ -240,7 +244,8 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
       const uint16_t* q_row = q + flat * d;
       const uint16_t* k_head = k + ((int64_t)b * Hkv + hkv) * Lk * d;
       const uint16_t* v_head = v + ((int64_t)b * Hkv + hkv) * Lk * d;
-      lse[r] = attend_row(q_row, k_head, v_head, d, scale, &m, b, i, 0, Lk, s_buf, ok_buf,
+      const double slope = alibi_slopes ? alibi_slopes[hq] : 0.0;
+      lse[r] = attend_row(q_row, k_head, v_head, d, scale, &m, b, i, 0, Lk, slope, s_buf, ok_buf,
                           q_buf, o + r * d);
     }
     free(s_buf);
@@ -248,6 +253,26 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
     free(q_buf);
   }
   return err ? -2 : 0;
+}
+
+int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                     int Hkv, int Lq, int Lk, int d, double scale, int mask_kind, int window_l,
+                     int window_r, int draft_block, const int32_t* doc_ids,
+                     const int32_t* kv_lens, const int64_t* rows, int64_t nrows, double* o,
+                     double* lse, int nthreads) {
+  return attn_rows(q, k, v, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
+                   draft_block, doc_ids, kv_lens, NULL, rows, nrows, o, lse, nthreads);
+}
+
+/* The same with the ALiBi score_mod: alibi_slopes[hq] per query head. */
+int oracle_attn_rows_alibi(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                           int Hq, int Hkv, int Lq, int Lk, int d, double scale, int mask_kind,
+                           int window_l, int window_r, int draft_block, const int32_t* doc_ids,
+                           const double* alibi_slopes, const int64_t* rows, int64_t nrows,
+                           double* o, double* lse, int nthreads) {
+  if (!alibi_slopes) return -1;
+  return attn_rows(q, k, v, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
+                   draft_block, doc_ids, NULL, alibi_slopes, rows, nrows, o, lse, nthreads);
 }
 
 /*
@@ -300,7 +325,7 @@ int oracle_decode_partials(const uint16_t* q, const uint16_t* k, const uint16_t*
         lse_part[(int64_t)s * nrows + r] =
             attend_row(q + r * d, k + ((int64_t)b * Hkv + hkv) * Lk * d,
                        v + ((int64_t)b * Hkv + hkv) * Lk * d, d, scale, &m, b, i, j_lo, j_hi,
-                       s_buf, ok_buf, q_buf, o_row);
+                       0.0, s_buf, ok_buf, q_buf, o_row);
       }
     }
     free(s_buf);

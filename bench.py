@@ -228,6 +228,25 @@ def run_prefill(cfg, timer, steps, warmup, stream, batch_mult=1):
     return c, inp, ms, algorithmic_flops(c, pairs)
 
 
+def run_alibi(cfg, timer, steps, warmup, stream):
+    """The headline workload with the ALiBi score_mod (slopes 2^(-8 (h+1) / H))."""
+    import sm_attn_fwd_b200 as ab
+    inp = make_inputs(cfg, device="cuda")
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / cfg.Hq) for h in range(cfg.Hq)],
+                          dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    o = torch.empty_like(inp.q)
+    lse = torch.empty(cfg.B, cfg.Hq, cfg.Lq, dtype=torch.float32, device="cuda")
+    fn = lambda: ab.attn_fwd_score_mod(inp.q, inp.k, inp.v, alibi_slopes=slopes,  # noqa: E731
+                                       scale=cfg.softmax_scale, mask=cfg.mask, o=o, lse=lse,
+                                       stream=stream)
+    ms = timer.time(fn, steps, warmup)
+    st, bits = ab.attn_get_device_error(stream)
+    if st != ab.ATTN_OK:
+        raise RuntimeError(f"device error after {cfg.name} with ALiBi: {st} {bits}")
+    return ms, algorithmic_flops(cfg, visible_pairs(cfg))
+
+
 # Packed sequences: 16 documents with lengths drawn uniformly from [128, 4096]
 # (seed 5), self-attention, causal, H = 16, d = 64.
 VARLEN_NAME = "varlen_causal_16seqs_l128to4096_h16_d64"
@@ -495,6 +514,13 @@ def main():
                 workloads[c2.name] = {"ms_median": med, "ms_min": min(ms2), "TFLOP/s": tf,
                                       "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
                                       "algorithmic_flop": fl2}
+            ms6, fl6 = run_alibi(HEADLINE, timer, max(5, args.steps // 10), 3, stream)
+            med = statistics.median(ms6)
+            tf = fl6 / (med * 1e9)
+            workloads[HEADLINE.name + "_alibi"] = {"ms_median": med, "ms_min": min(ms6),
+                                                   "TFLOP/s": tf,
+                                                   "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
+                                                   "algorithmic_flop": fl6}
             ms5, fl5, lens5 = run_varlen(timer, max(5, args.steps // 10), 3, stream)
             med = statistics.median(ms5)
             tf = fl5 / (med * 1e9)

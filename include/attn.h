@@ -92,6 +92,33 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        int window_l, int window_r, int draft_block, const int32_t* doc_ids,
                        void* stream);
 
+typedef enum {
+  ATTN_SCORE_MOD_NONE = 0,  /* S_ij unchanged */
+  ATTN_SCORE_MOD_ALIBI = 1  /* S_ij += slope[hq] * (j - p); params = slope[Hq] */
+} attn_score_mod_kind_t;
+
+/*
+ * attn_fwd_score_mod — attn_fwd with a score modifier.
+ *
+ * Defines ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", section 1:
+ * score_mod(score, b, h, q_idx, kv_idx) -> score, e.g. ALiBi or a position
+ * bias): the scaled score S_ij of attn_fwd is replaced by the modified score
+ * before the mask and the softmax; LSE is taken over the modified scores.
+ *   ATTN_SCORE_MOD_ALIBI: S_ij = scale * <Q_i, K_j> + slope[hq] * (j - p), with
+ *   p = Lk - Lq + i the row's absolute position and slope a caller-given
+ *   per-query-head value (for example 2^(-8 (hq+1) / Hq)).
+ *
+ * Arguments: those of attn_fwd, plus
+ *   score_mod         one of attn_score_mod_kind_t
+ *   score_mod_params  ALIBI: [Hq] fp32 device array (4-byte aligned); NONE: ignored
+ * Errors: as attn_fwd; INVALID_ARG for an unknown score_mod or missing params.
+ */
+attn_status_t attn_fwd_score_mod(const void* q, const void* k, const void* v, void* o,
+                                 float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                                 float scale, int mask_kind, int window_l, int window_r,
+                                 int draft_block, const int32_t* doc_ids, int score_mod,
+                                 const float* score_mod_params, void* stream);
+
 /*
  * attn_fwd_varlen — prefill attention forward over packed sequences.
  *

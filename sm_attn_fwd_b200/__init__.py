@@ -25,7 +25,8 @@ __all__ = [
     "AttnError", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
-    "attn_fwd", "attn_fwd_varlen", "attn_decode_splitkv", "attn_decode_num_splits",
+    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_decode_splitkv",
+    "attn_decode_num_splits", "SCORE_MOD_NONE", "SCORE_MOD_ALIBI",
     "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
     "EXPORTED_SYMBOLS",
@@ -41,10 +42,13 @@ ATTN_ERR_TIMEOUT = 5
 MASK_NONE = 0
 MASK_CAUSAL = 1
 MASK_DRAFT_BLOCK = 2
+SCORE_MOD_NONE = 0
+SCORE_MOD_ALIBI = 1
 _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 
 EXPORTED_SYMBOLS = (
-    "attn_fwd", "attn_fwd_varlen", "attn_decode_num_splits", "attn_decode_workspace_size",
+    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_decode_num_splits",
+    "attn_decode_workspace_size",
     "attn_decode_splitkv", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
 )
@@ -79,6 +83,9 @@ def load_library():
         lib.attn_fwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, i32,
                                  i32, P, P]
         lib.attn_fwd.restype = i32
+        lib.attn_fwd_score_mod.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
+                                           i32, i32, i32, P, i32, P, P]
+        lib.attn_fwd_score_mod.restype = i32
         lib.attn_fwd_varlen.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32,
                                         i32, i32, i32, i32, P]
         lib.attn_fwd_varlen.restype = i32
@@ -154,6 +161,37 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
                                  int(draft_block), _ptr(doc_ids), _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_score_mod(q, k, v, *, alibi_slopes, scale=None, mask="none", window=(-1, -1),
+                       draft_block=1, doc_ids=None, o=None, lse=None, stream=None):
+    """attn_fwd with the ALiBi score_mod (see ``attn_fwd_score_mod`` in include/attn.h):
+    S_ij += alibi_slopes[hq] * (j - p).  alibi_slopes: fp32 CUDA tensor [Hq]."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_bf16(name, t)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    if (alibi_slopes.dtype != torch.float32 or not alibi_slopes.is_cuda
+            or not alibi_slopes.is_contiguous() or alibi_slopes.numel() != Hq):
+        raise ValueError("alibi_slopes must be a contiguous fp32 CUDA tensor [Hq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    if doc_ids is not None:
+        if doc_ids.dtype != torch.int32 or not doc_ids.is_cuda or not doc_ids.is_contiguous():
+            raise ValueError("doc_ids must be a contiguous int32 CUDA tensor [B, Lk]")
+    mk = mask if isinstance(mask, int) else _MASKS[mask]
+    st = load_library().attn_fwd_score_mod(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
+                                           Hkv, Lq, Lk, d, float(scale), mk, int(window[0]),
+                                           int(window[1]), int(draft_block), _ptr(doc_ids),
+                                           SCORE_MOD_ALIBI, _ptr(alibi_slopes),
+                                           _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_score_mod")
     return o, lse
 
 

@@ -167,10 +167,10 @@ const char* attn_status_string(attn_status_t s) {
   return "ATTN_ERR_UNKNOWN";
 }
 
-attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                       int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_kind,
-                       int window_l, int window_r, int draft_block, const int32_t* doc_ids,
-                       void* stream) {
+static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                               int mask_kind, int window_l, int window_r, int draft_block,
+                               const int32_t* doc_ids, const float* alibi_slopes, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4))
@@ -190,6 +190,7 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.o = o;
   p.lse = lse;
   p.doc_ids = doc_ids;
+  p.alibi_slopes = alibi_slopes;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -219,6 +220,28 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
   cudaError_t e = d == 64 ? attn::launch_prefill<64>(tq, tk, tv, p, grid, st)
                           : attn::launch_prefill<128>(tq, tk, tv, p, grid, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                       int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_kind,
+                       int window_l, int window_r, int draft_block, const int32_t* doc_ids,
+                       void* stream) {
+  return fwd_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
+                   draft_block, doc_ids, nullptr, stream);
+}
+
+attn_status_t attn_fwd_score_mod(const void* q, const void* k, const void* v, void* o,
+                                 float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                                 float scale, int mask_kind, int window_l, int window_r,
+                                 int draft_block, const int32_t* doc_ids, int score_mod,
+                                 const float* score_mod_params, void* stream) {
+  if (score_mod == ATTN_SCORE_MOD_NONE)
+    return fwd_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
+                     draft_block, doc_ids, nullptr, stream);
+  if (score_mod != ATTN_SCORE_MOD_ALIBI) return ATTN_ERR_INVALID_ARG;
+  if (!score_mod_params || !aligned(score_mod_params, 4)) return ATTN_ERR_INVALID_ARG;
+  return fwd_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
+                   draft_block, doc_ids, score_mod_params, stream);
 }
 
 attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

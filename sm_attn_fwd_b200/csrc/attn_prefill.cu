@@ -39,11 +39,12 @@ namespace attn {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kRegsLow = 72;    // warpgroup 0 (producer, MMA)
-constexpr int kRegsHigh = 216;  // softmax warpgroups: 72*128 + 2*216*128 = 168*384
+constexpr int kRegsLow = 80;    // warpgroup 0 (producer, MMA)
+constexpr int kRegsHigh = 208;  // softmax warpgroups: 80*128 + 2*208*128 <= 168*384
 constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
+constexpr float kLog2e = 1.44269504088896340736f;
 constexpr int kBitWords = kMaxKvTiles / 32;
 
 struct Sched {
@@ -327,7 +328,9 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile_saddr, int kk) {
 
 }  // namespace
 
-template <int D>
+// kAlibi: the ALiBi score_mod, S_ij += slope_h * (j - p) (p the row's absolute
+// position), with p.alibi_slopes[hq] per query head.
+template <int D, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -716,6 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_o_done = BAR(kODone + x);
     const uint32_t bar_o_free = BAR(kOFree + x);
     const float c = p.scale_log2;
+    const float c_s = kAlibi ? 1.0f : c;  // scale still to apply to the loaded scores
     int ns = 0;  // S tiles consumed (global count)
     // The two softmax warpgroups take turns on the exponentials of each key
     // tile (A, B, A, B, ...), so that one loads S, finds the row max and stores
@@ -737,6 +741,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       const bool row_ok = r_row < w.rows[x];
+      // ALiBi: the row's absolute position and the head's slope times log2(e)
+      const long long row_pos = w.pos0[x] + r_row;
+      const float alibi2 = kAlibi ? __ldg(p.alibi_slopes + w.hq) * kLog2e : 0.0f;
       int row_lo = 0, row_hi = -1;  // visible key range, clamped to [0, Lk-1]
       int row_doc = 0;
       // document ids of this batch row (warp-uniform: every lane takes part in
@@ -857,6 +864,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[i] = ((word >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
           }
         }
+        if constexpr (kAlibi) {
+          // scores to the base-2 domain with the bias: s*c + slope*log2(e)*(j - p);
+          // masked scores stay -inf.  The max and the exponentials below then
+          // use a scale of 1.
+          const float base = alibi2 * (float)(k0 - row_pos);
+#pragma unroll
+          for (int i = 0; i < 128; ++i) sv[i] = fmaf(sv[i], c, fmaf(alibi2, (float)i, base));
+        }
         // row max: sixteen independent chains of two-input max, then a tree
         float mx16[16];
 #pragma unroll
@@ -872,7 +887,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < w; ++j) mx16[j] = fmaxf(mx16[j], mx16[j + w]);
         }
         const float mx = mx16[0];
-        const float m_new = fmaxf(m_ref, mx * c);
+        const float m_new = fmaxf(m_ref, mx * c_s);
         const bool need = m_new > m_ref + kRescaleThreshold;
         const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;
         if (need) {
@@ -910,7 +925,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i < 64) {
               const int i0 = 2 * i, i1 = i0 + 1;
               float a0, a1;
-              ptx::fma2_bc(a0, a1, sv[i0], sv[i1], c, -m_use);  // s * c - m, two at once
+              ptx::fma2_bc(a0, a1, sv[i0], sv[i1], c_s, -m_use);  // s * c - m, two at once
               e0[i % kAhead] = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
               e1[i % kAhead] = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
             }
@@ -1028,10 +1043,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
-cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           const FwdParams& p, int grid, cudaStream_t stream) {
-  auto kern = attn_prefill_kernel<D>;
+template <int D, bool kAlibi>
+cudaError_t launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tk,
+                                  const CUtensorMap& tv, const FwdParams& p, int grid,
+                                  cudaStream_t stream) {
+  auto kern = attn_prefill_kernel<D, kAlibi>;
   constexpr int smem = Cfg<D>::kSmemAlloc;
   static bool configured[64] = {};
   int dev = 0;
@@ -1045,6 +1061,13 @@ cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const C
   }
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           const FwdParams& p, int grid, cudaStream_t stream) {
+  return p.alibi_slopes ? launch_prefill_kernel<D, true>(tq, tk, tv, p, grid, stream)
+                        : launch_prefill_kernel<D, false>(tq, tk, tv, p, grid, stream);
 }
 
 template cudaError_t launch_prefill<64>(const CUtensorMap&, const CUtensorMap&,

@@ -136,3 +136,16 @@ def test_attn_fwd_varlen_rejects_on_host():
     assert call(a15=2, a18=0) == ab.ATTN_ERR_INVALID_ARG   # draft block < 1
     assert call(a16=-2) == ab.ATTN_ERR_INVALID_ARG         # window < -1
     assert call(a13=96) == ab.ATTN_ERR_UNSUPPORTED         # d
+
+
+def test_attn_fwd_score_mod_rejects_on_host():
+    lib = ab.load_library()
+    #      q  k  v  o  lse B  Hq Hkv Lq   Lk   d   scale mask wl  wr bd doc  kind params stream
+    args = [A, A, A, A, A, 2, 8, 2, 100, 100, 64, 0.125, 1, -1, -1, 1, None, 1, A, None]
+    assert lib.attn_fwd_score_mod(*args[:17], 7, A, None) == ab.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_score_mod(*args[:17], 1, None, None) == ab.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_score_mod(*args[:17], 1, ctypes.c_void_p(0x10002), None) == \
+        ab.ATTN_ERR_INVALID_ARG
+    bad_d = list(args)
+    bad_d[10] = 96
+    assert lib.attn_fwd_score_mod(*bad_d) == ab.ATTN_ERR_UNSUPPORTED

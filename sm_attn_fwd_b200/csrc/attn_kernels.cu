@@ -52,7 +52,7 @@ struct Cfg {
   static constexpr int kAtoms = D / 64;               // 128-byte swizzle atoms along d
   static constexpr int kAtomBytes = kBlockN * 128;    // one atom column of a 128-row tile
   static constexpr int kTileBytes = kBlockN * D * 2;  // one K or V tile (== Q tile)
-  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kStages = (D == 64) ? 4 : 3;  // d = 128: 3 x 64 KB of K/V, 226 KB in all
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;

@@ -146,8 +146,8 @@ __device__ __forceinline__ float exp2_fma(float x) {
 
 // Which of the 128 exponentials of a row go to the FMA pipe.  Measured on
 // B200 (causal 4K d=64 and 32K d=128): any share made the kernel slower
-// (1/8: -4%, 2/8: -7%), since the softmax is bound by instruction issue and
-// handoff latency, not by the MUFU unit; kept switched off.
+// (1/16: -1%, 1/8: -7%, 1/4: -10%), since the softmax is not limited by MUFU
+// throughput alone; kept switched off.
 constexpr bool kExpFmaShare = false;
 __host__ __device__ constexpr bool exp_on_fma(int i) { return (i & 7) == 3 && kExpFmaShare; }
 

@@ -14,9 +14,9 @@
 #include "attn_params.h"
 
 namespace attn {
-template <int D, bool kDecode>
-cudaError_t launch_fwd(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                       const FwdParams&, dim3, cudaStream_t);
+template <int D>
+cudaError_t launch_decode(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                          const FwdParams&, dim3, cudaStream_t);
 template <int D>
 cudaError_t launch_combine(const FwdParams&, cudaStream_t);
 template <int D>
@@ -391,8 +391,8 @@ attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cach
 
   dim3 grid((unsigned)pl.nsplit, (unsigned)(B * Hkv * pl.row_tiles), 1);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = d == 64 ? attn::launch_fwd<64, true>(tq, tk, tv, p, grid, st)
-                          : attn::launch_fwd<128, true>(tq, tk, tv, p, grid, st);
+  cudaError_t e = d == 64 ? attn::launch_decode<64>(tq, tk, tv, p, grid, st)
+                          : attn::launch_decode<128>(tq, tk, tv, p, grid, st);
   if (e != cudaSuccess) return ATTN_ERR_CUDA;
   e = d == 64 ? attn::launch_combine<64>(p, st) : attn::launch_combine<128>(p, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

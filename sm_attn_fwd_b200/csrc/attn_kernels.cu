@@ -1,16 +1,15 @@
-// Fused tiled attention forward for sm_100a (B200): prefill and split-KV decode.
+// Split-KV decode for sm_100a (B200): the partial kernel and the combine.
+// (The prefill forward is the persistent kernel in attn_prefill.cu.)
 //
 // Method ("FlashAttention 2 原理与 PyTorch 实战", sections 一, 3.1, 3.2): a CTA owns
 // one 128-row query tile, streams 128-key K/V tiles through shared memory,
 // computes S = Q K^T, applies the mask, keeps a running row max m and sum l
 // (online softmax), rescales the accumulator and adds P V, so the N x N score
-// matrix never reaches HBM.  The mask is the mask_mod predicate of
-// "FlexAttention 是什么，以及 DFlash2 之谜的完整侦破" (section 1: causal, sliding
-// window, non-causal, document ids; section 3: the symmetric window and the
-// block-diffusion draft mask).  The split-KV decode (same page, section 1,
-// FlexDecoding / FlashDecoding) gives each CTA one chunk of the KV cache and
-// leaves a normalised partial output plus its log-sum-exp for the combine
-// kernel at the end of this file.
+// matrix never reaches HBM.  The split-KV decode ("FlexAttention 是什么，以及
+// DFlash2 之谜的完整侦破", section 1, FlexDecoding / FlashDecoding) gives each CTA
+// one chunk of the KV cache of one sequence (every query row sees the keys
+// [0, kv_lens[b]) of its sequence) and leaves a normalised partial output plus
+// its log-sum-exp for the combine kernel at the end of this file.
 //
 // B200 mapping (one CTA per SM, 192 threads):
 //   warp 0      TMA producer: Q once, then K and V tiles into a ring of stages
@@ -75,26 +74,6 @@ struct Misc {
   int t_hi;
 };
 
-__device__ __forceinline__ long long floor_div_ll(long long a, long long b) {
-  return a >= 0 ? a / b : -((-a + b - 1) / b);
-}
-
-// Inclusive key range [lo, hi] the mask allows for a query at absolute
-// position pos, before the document test.  hi < lo means none.
-__device__ __forceinline__ void key_bounds(const FwdParams& p, long long pos, long long& lo,
-                                           long long& hi) {
-  lo = 0;
-  hi = (long long)p.Lk - 1;
-  if (p.mask_kind == kMaskCausal) {
-    hi = min(hi, pos);
-  } else if (p.mask_kind == kMaskDraftBlock) {
-    long long bd = p.draft_block;
-    hi = min(hi, (floor_div_ll(pos, bd) + 1) * bd - 1);
-  }
-  if (p.window_l >= 0) lo = max(lo, pos - (long long)p.window_l);
-  if (p.window_r >= 0) hi = min(hi, pos + (long long)p.window_r);
-}
-
 __device__ __forceinline__ bool bit_get(const uint32_t* bits, int i) {
   return (bits[i >> 5] >> (i & 31)) & 1u;
 }
@@ -116,9 +95,9 @@ __device__ __forceinline__ uint64_t desc_v_mnmajor(uint32_t tile_saddr, int kk) 
 
 }  // namespace
 
-template <int D, bool kDecode>
+template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q,
+    attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = Cfg<D>;
@@ -148,58 +127,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
 
   // ------------------------------------------------------------ work unit
-  int b, hkv, rows_valid, kv_z, q_coord_y, q_coord_z;
-  long long pos0 = 0;      // absolute position of tile row 0 (prefill)
-  int key_end;             // keys at or past this index are never visible
-  int t_lo, t_hi;          // candidate key tiles (absolute tile indices)
-  long long row_out0;      // flat output row of tile row 0
-  int split = 0;
-  if constexpr (kDecode) {
-    split = blockIdx.x;
-    const int bh = blockIdx.y / p.row_tiles;
-    const int rt = blockIdx.y % p.row_tiles;
-    b = bh / p.Hkv;
-    hkv = bh % p.Hkv;
-    int kv_len = p.kv_lens[b];
-    if (kv_len < 0 || kv_len > p.Lk) {
-      if (threadIdx.x == 0 && blockIdx.x == 0 && rt == 0) atomicOr(&g_device_error, kDevErrBadKvLen);
-      kv_len = kv_len < 0 ? 0 : p.Lk;
-    }
-    const int c0 = split * p.chunk;
-    if (c0 >= kv_len) return;  // this split holds no keys of sequence b (uniform exit)
-    key_end = min(c0 + p.chunk, kv_len);
-    rows_valid = min(kBlockM, p.group * p.Lq - rt * kBlockM);
-    row_out0 = ((long long)b * p.Hq + (long long)hkv * p.group) * p.Lq + (long long)rt * kBlockM;
-    q_coord_y = (int)row_out0;
-    q_coord_z = 0;
-    kv_z = b * p.Hkv + hkv;
-    t_lo = c0 / kBlockN;
-    t_hi = (key_end - 1) / kBlockN;
-  } else {
-    const int qt = p.q_tiles - 1 - (int)blockIdx.x;  // heaviest causal tiles first
-    const int bhq = blockIdx.y;
-    b = bhq / p.Hq;
-    const int hq = bhq % p.Hq;
-    hkv = hq / p.group;
-    const int q0 = qt * kBlockM;
-    rows_valid = min(kBlockM, p.Lq - q0);
-    row_out0 = (long long)bhq * p.Lq + q0;
-    q_coord_y = q0;
-    q_coord_z = bhq;
-    kv_z = b * p.Hkv + hkv;
-    key_end = p.Lk;
-    pos0 = (long long)p.Lk - p.Lq + q0;
-    long long lo_a, hi_a, lo_b, hi_b;
-    key_bounds(p, pos0, lo_a, hi_a);
-    key_bounds(p, pos0 + rows_valid - 1, lo_b, hi_b);
-    if (hi_b < lo_a || hi_b < 0) {
-      t_lo = 0;
-      t_hi = -1;
-    } else {
-      t_lo = (int)(lo_a / kBlockN);
-      t_hi = (int)(hi_b / kBlockN);
-    }
+  // (split, b, kv head, 128-row tile of the group's Hq/Hkv x Lq query rows)
+  const int split = blockIdx.x;
+  const int bh = blockIdx.y / p.row_tiles;
+  const int rt = blockIdx.y % p.row_tiles;
+  const int b = bh / p.Hkv;
+  const int hkv = bh % p.Hkv;
+  int kv_len = p.kv_lens[b];
+  if (kv_len < 0 || kv_len > p.Lk) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && rt == 0) atomicOr(&g_device_error, kDevErrBadKvLen);
+    kv_len = kv_len < 0 ? 0 : p.Lk;
   }
+  const int c0 = split * p.chunk;
+  if (c0 >= kv_len) return;  // this split holds no keys of sequence b (uniform exit)
+  const int key_end = min(c0 + p.chunk, kv_len);  // keys at or past this are never visible
+  const int rows_valid = min(kBlockM, p.group * p.Lq - rt * kBlockM);
+  // flat output row of tile row 0
+  const long long row_out0 =
+      ((long long)b * p.Hq + (long long)hkv * p.group) * p.Lq + (long long)rt * kBlockM;
+  const int q_coord_y = (int)row_out0;
+  const int kv_z = b * p.Hkv + hkv;
+  const int t_lo = c0 / kBlockN;  // candidate key tiles (absolute tile indices)
+  const int t_hi = (key_end - 1) / kBlockN;
 
   // ------------------------------------------------------------- prologue
   if (warp == 0) {
@@ -226,68 +175,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       misc->t_hi = t_hi;
       ptx::fence_mbar_init();
     }
-    // Tile classification: EMPTY tiles are skipped, FULL tiles need no mask.
+    // Tile classification: FULL tiles lie below kv_len and need no mask.
     const int ntc = t_hi - t_lo + 1;
     int n_tiles = 0;
-    int qdmin = 0, qdmax = 0;
-    const int32_t* doc_b = nullptr;
-    if (!kDecode && p.doc_ids != nullptr && ntc > 0) {
-      doc_b = p.doc_ids + (long long)b * p.Lk;
-      int mn = 0x7fffffff, mx = (int)0x80000000;
-      for (int r = lane; r < rows_valid; r += 32) {
-        const int d = __ldg(doc_b + (pos0 + r));
-        mn = min(mn, d);
-        mx = max(mx, d);
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
-      qdmin = mn;
-      qdmax = mx;
-    }
-    long long lo_b = 0, hi_a = -1;
-    if (!kDecode) {
-      long long lo_a, hi_b;
-      key_bounds(p, pos0, lo_a, hi_a);
-      key_bounds(p, pos0 + rows_valid - 1, lo_b, hi_b);
-    }
     for (int base = 0; base < ntc; base += 32) {
       const int i = base + lane;
-      const int t = t_lo + i;
-      bool empty = false, full = false;
-      if (i < ntc) {
-        const long long k0 = (long long)t * kBlockN;
-        if constexpr (kDecode) {
-          full = (k0 + kBlockN <= key_end);
-        } else {
-          full = (k0 + kBlockN <= p.Lk) && (lo_b <= k0) && (hi_a >= k0 + kBlockN - 1);
-        }
-      }
-      if (doc_b != nullptr) {
-        // document ids: per tile min/max over the tile's keys (whole warp per tile)
-        for (int w = 0; w < 32 && base + w < ntc; ++w) {
-          const long long k0 = (long long)(t_lo + base + w) * kBlockN;
-          const int kend = (int)min(k0 + kBlockN, (long long)p.Lk);
-          int mn = 0x7fffffff, mx = (int)0x80000000;
-          for (long long kk = k0 + lane; kk < kend; kk += 32) {
-            const int d = __ldg(doc_b + kk);
-            mn = min(mn, d);
-            mx = max(mx, d);
-          }
-          for (int o = 16; o > 0; o >>= 1) {
-            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          }
-          if (lane == w) {
-            if (mx < qdmin || mn > qdmax) empty = true;
-            if (!(mn == mx && qdmin == qdmax && mn == qdmin)) full = false;
-          }
-        }
-      }
-      if (i >= ntc) empty = true;
+      const long long k0 = (long long)(t_lo + i) * kBlockN;
+      const bool empty = i >= ntc;
+      const bool full = !empty && (k0 + kBlockN <= key_end);
       const uint32_t eb = __ballot_sync(0xffffffffu, empty);
-      const uint32_t fb = __ballot_sync(0xffffffffu, full && !empty);
+      const uint32_t fb = __ballot_sync(0xffffffffu, full);
       if (lane == 0) {
         empty_bits[base >> 5] = eb;
         full_bits[base >> 5] = fb;
@@ -313,13 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t kTx = C::kTileBytes;
       if (lane == 0) {
         ptx::mbar_arrive_expect_tx(q_full, kTx);
-        for (int a = 0; a < C::kAtoms; ++a) {
-          if constexpr (kDecode)
-            ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y);
-          else
-            ptx::tma_load_3d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y,
-                             q_coord_z);
-        }
+        for (int a = 0; a < C::kAtoms; ++a)
+          ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y);
       }
       // One 128-key K or V tile into shared memory.  Contiguous cache: one box
       // per 64-column atom.  Paged cache ([num_pages, Hkv, page_size, d] through
@@ -462,23 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_ok = r < rows_valid;
     const float c = p.scale_log2;
 
-    // visible key range of this row, before the document test
-    long long row_lo = 0, row_hi = -1;
-    int row_doc = 0;
-    const int32_t* doc_b = nullptr;
-    if (row_ok) {
-      if constexpr (kDecode) {
-        row_lo = 0;
-        row_hi = key_end - 1;
-      } else {
-        const long long pos = pos0 + r;
-        key_bounds(p, pos, row_lo, row_hi);
-        if (p.doc_ids != nullptr) {
-          doc_b = p.doc_ids + (long long)b * p.Lk;
-          row_doc = __ldg(doc_b + pos);
-        }
-      }
-    }
+    // every query row of the sequence sees the keys [0, kv_len); rows past the
+    // tile's valid rows see none
+    const long long row_hi = row_ok ? (long long)key_end - 1 : -1;
 
     float m_ref = -INFINITY;  // reference max (base-2 scaled units)
     float l = 0.0f;
@@ -508,10 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!full) {
 #pragma unroll
         for (int i = 0; i < kBlockN; ++i) {
-          const long long key = k0 + i;
-          bool vis = (key >= row_lo) && (key <= row_hi);
-          if (doc_b != nullptr && vis) vis = (__ldg(doc_b + key) == row_doc);
-          s[i] = vis ? s[i] : -INFINITY;
+          s[i] = (k0 + i <= row_hi) ? s[i] : -INFINITY;
         }
       }
       float mx = -INFINITY;
@@ -557,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_st32(t_row + tmem_s(j) + h * 32, packed);
       }
       l += rowsum;
-      if constexpr (kDecode) {
+      {
         // Keys past the end of this sequence: their V rows may hold anything
         // (even NaN), and 0 * NaN would poison O.  Zero them in shared memory.
         if (!full) {
@@ -609,40 +484,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < 32; ++i) raw[i] = 0u;
       }
       if (row_ok) {
-        if constexpr (kDecode) {
-          float* dst = p.ws_o + ((long long)split * p.B * p.Hq * p.Lq + out_row) * D + cc * 32;
+        float* dst = p.ws_o + ((long long)split * p.B * p.Hq * p.Lq + out_row) * D + cc * 32;
 #pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            float4 v4 = make_float4(__uint_as_float(raw[i]) * inv_l,
-                                    __uint_as_float(raw[i + 1]) * inv_l,
-                                    __uint_as_float(raw[i + 2]) * inv_l,
-                                    __uint_as_float(raw[i + 3]) * inv_l);
-            *reinterpret_cast<float4*>(dst + i) = v4;
-          }
-        } else {
-          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + out_row * D + cc * 32;
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            uint4 v4;
-            v4.x = ptx::pack_bf16x2(__uint_as_float(raw[i]) * inv_l,
-                                    __uint_as_float(raw[i + 1]) * inv_l);
-            v4.y = ptx::pack_bf16x2(__uint_as_float(raw[i + 2]) * inv_l,
-                                    __uint_as_float(raw[i + 3]) * inv_l);
-            v4.z = ptx::pack_bf16x2(__uint_as_float(raw[i + 4]) * inv_l,
-                                    __uint_as_float(raw[i + 5]) * inv_l);
-            v4.w = ptx::pack_bf16x2(__uint_as_float(raw[i + 6]) * inv_l,
-                                    __uint_as_float(raw[i + 7]) * inv_l);
-            *reinterpret_cast<uint4*>(dst + i) = v4;
-          }
+        for (int i = 0; i < 32; i += 4) {
+          float4 v4 = make_float4(__uint_as_float(raw[i]) * inv_l,
+                                  __uint_as_float(raw[i + 1]) * inv_l,
+                                  __uint_as_float(raw[i + 2]) * inv_l,
+                                  __uint_as_float(raw[i + 3]) * inv_l);
+          *reinterpret_cast<float4*>(dst + i) = v4;
         }
       }
     }
-    if (row_ok) {
-      if constexpr (kDecode)
-        p.ws_lse[(long long)split * p.B * p.Hq * p.Lq + out_row] = lse_row;
-      else
-        p.lse[out_row] = lse_row;
-    }
+    if (row_ok) p.ws_lse[(long long)split * p.B * p.Hq * p.Lq + out_row] = lse_row;
   }
 
   // ------------------------------------------------------------- teardown
@@ -734,10 +587,10 @@ cudaError_t launch_selftest_wait(cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------- launchers
-template <int D, bool kDecode>
-cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const FwdParams& p, dim3 grid, cudaStream_t stream) {
-  auto kern = attn_fwd_kernel<D, kDecode>;
+template <int D>
+cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const FwdParams& p, dim3 grid, cudaStream_t stream) {
+  auto kern = attn_decode_kernel<D>;
   constexpr int smem = Cfg<D>::kSmemAlloc;
   // The shared-memory opt-in is set once per device, outside any stream capture
   // that a later call may be part of.
@@ -764,12 +617,10 @@ cudaError_t launch_combine(const FwdParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
-template cudaError_t launch_fwd<64, true>(const CUtensorMap&, const CUtensorMap&,
-                                          const CUtensorMap&, const FwdParams&, dim3,
-                                          cudaStream_t);
-template cudaError_t launch_fwd<128, true>(const CUtensorMap&, const CUtensorMap&,
-                                           const CUtensorMap&, const FwdParams&, dim3,
-                                           cudaStream_t);
+template cudaError_t launch_decode<64>(const CUtensorMap&, const CUtensorMap&,
+                                        const CUtensorMap&, const FwdParams&, dim3, cudaStream_t);
+template cudaError_t launch_decode<128>(const CUtensorMap&, const CUtensorMap&,
+                                         const CUtensorMap&, const FwdParams&, dim3, cudaStream_t);
 template cudaError_t launch_combine<64>(const FwdParams&, cudaStream_t);
 template cudaError_t launch_combine<128>(const FwdParams&, cudaStream_t);
 

@@ -868,9 +868,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           // scores to the base-2 domain with the bias: s*c + slope*log2(e)*(j - p);
           // masked scores stay -inf.  The max and the exponentials below then
           // use a scale of 1.
+          // The bias of key pair i (keys 2i, 2i+1) comes from one of eight chains
+          // that step 16 keys at a time: one packed add and one packed FMA per pair.
           const float base = alibi2 * (float)(k0 - row_pos);
+          const float step = alibi2 * 16.0f;
+          float b0[8], b1[8];
 #pragma unroll
-          for (int i = 0; i < 128; ++i) sv[i] = fmaf(sv[i], c, fmaf(alibi2, (float)i, base));
+          for (int k = 0; k < 8; ++k) {
+            b0[k] = fmaf(alibi2, (float)(2 * k), base);
+            b1[k] = fmaf(alibi2, (float)(2 * k + 1), base);
+          }
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int k = i & 7;
+            ptx::fma2_bv(sv[2 * i], sv[2 * i + 1], sv[2 * i], sv[2 * i + 1], c, b0[k], b1[k]);
+            if (i + 8 < 64) ptx::add2_acc(b0[k], b1[k], step, step);
+          }
         }
         // row max: sixteen independent chains of two-input max, then a tree
         float mx16[16];

@@ -413,6 +413,18 @@ __device__ __forceinline__ void fma2_bc(float& d0, float& d1, float a0, float a1
       : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 // (s0, s1) += (a0, a1)
+// (a0 * b + c0, a1 * b + c1) as one packed fp32x2 FMA.
+__device__ __forceinline__ void fma2_bv(float& d0, float& d1, float a0, float a1, float b,
+                                        float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %4};\n\t"
+      "mov.b64 rc, {%5, %6};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c0), "f"(c1));
+}
 __device__ __forceinline__ void add2_acc(float& s0, float& s1, float a0, float a1) {
   asm("{\n\t.reg .b64 rs, ra;\n\t"
       "mov.b64 rs, {%0, %1};\n\t"

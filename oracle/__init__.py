@@ -119,6 +119,9 @@ def mask(B, Lq, Lk, *, mask="none", window=(-1, -1), draft_block=1, doc_ids=None
     return out.astype(bool)
 
 
+_mask_matrix = mask  # the mask function above, for callers whose argument is named `mask`
+
+
 def count_pairs(B, Lq, Lk, *, mask="none", window=(-1, -1), draft_block=1, doc_ids=None,
                 kv_lens=None, nthreads=None) -> int:
     """Allowed (query row, key) pairs summed over the batch, for ONE head."""
@@ -273,3 +276,55 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale=None, mask="no
         o[q0:q1] = ob[0].transpose(1, 0, 2)
         lse[:, q0:q1] = lb[0]
     return o, lse
+
+
+def attn_bwd(q, k, v, do, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
+             doc_ids=None):
+    """Gradients of the forward above: (dQ, dK, dV) in double, for bf16 inputs.
+
+    The backward of softmax attention ("FlashAttention 2 原理与 PyTorch 实战",
+    section 3.2: the row statistics of the forward are recomputed, not stored
+    as an N x N matrix), written out on whole score rows: with P the masked
+    softmax of S = scale * Q K^T and O = P V,
+        dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,
+        dS = P * (dP - D),  dQ = scale * dS K,  dK = scale * dS^T Q.
+    Rows with no visible key have P = 0 and contribute nothing.  Query heads of
+    one KV head (GQA) add their dK and dV.  q: [B, Hq, Lq, d]; k, v: [B, Hkv, Lk, d];
+    do: [B, Hq, Lq, d] (any float dtype, read as double).  Returns float64 numpy
+    arrays shaped like q, k, v.
+    """
+    def as_f64(t):
+        if isinstance(t, np.ndarray):
+            return t.astype(np.float64)
+        return t.detach().cpu().double().numpy()
+
+    Q, K, V, dO = as_f64(q), as_f64(k), as_f64(v), as_f64(do)
+    B, Hq, Lq, d = Q.shape
+    _, Hkv, Lk, _ = K.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    group = Hq // Hkv
+    allowed = _mask_matrix(B, Lq, Lk, mask=mask, window=window, draft_block=draft_block,
+                           doc_ids=doc_ids)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    for b in range(B):
+        vis = allowed[b]
+        for hq in range(Hq):
+            hk = hq // group
+            S = scale * Q[b, hq] @ K[b, hk].T
+            S = np.where(vis, S, -np.inf)
+            mx = S.max(axis=1, keepdims=True)
+            has = np.isfinite(mx)
+            E = np.where(vis, np.exp(S - np.where(has, mx, 0.0)), 0.0)
+            l = E.sum(axis=1, keepdims=True)
+            P = np.where(has, E / np.where(l > 0, l, 1.0), 0.0)
+            O = P @ V[b, hk]
+            dV[b, hk] += P.T @ dO[b, hq]
+            dP = dO[b, hq] @ V[b, hk].T
+            Dv = (dO[b, hq] * O).sum(axis=1, keepdims=True)
+            dS = P * (dP - Dv)
+            dQ[b, hq] = scale * dS @ K[b, hk]
+            dK[b, hk] += scale * dS.T @ Q[b, hq]
+    return dQ, dK, dV

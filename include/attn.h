@@ -155,6 +155,43 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
                               int draft_block, void* stream);
 
 /*
+ * attn_bwd_workspace_size — bytes of caller workspace attn_bwd needs:
+ * an fp32 dQ accumulator [B, Hq, Lq, d] (rounded up to 256 bytes), then fp32
+ * D [B, Hq, Lq].  0 for invalid arguments.
+ */
+size_t attn_bwd_workspace_size(int B, int Hq, int Lq, int d);
+
+/*
+ * attn_bwd — gradients of attn_fwd: dQ, dK, dV for a given dO.
+ *
+ * Defines (the gradient of the definition above; "FlashAttention 2 原理与
+ * PyTorch 实战", section 3.2: the scores are recomputed from Q, K and the
+ * forward's LSE rather than stored): with P_ij = exp(S_ij - LSE_i) over the
+ * visible keys (0 elsewhere and for rows with no visible key),
+ *   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,  dS = P (dP - D),
+ *   dQ = scale dS K,  dK = scale dS^T Q,
+ * with the dK and dV of a KV head summed over its query heads (GQA).
+ *
+ * Arguments
+ *   q, o, dout  [B, Hq, Lq, d] bf16, read (o and lse from attn_fwd)
+ *   lse      [B, Hq, Lq] fp32, read
+ *   k, v     [B, Hkv, Lk, d] bf16, read
+ *   dq       [B, Hq, Lq, d] bf16, written;  dk, dv  [B, Hkv, Lk, d] bf16, written
+ *   B, Hq, Hkv, Lq, Lk, scale, mask_kind, window_l, window_r, draft_block,
+ *   doc_ids  as for attn_fwd; d = 64 (else UNSUPPORTED)
+ *   workspace  device memory, 256-byte aligned, >= attn_bwd_workspace_size bytes,
+ *            owned by the caller, not shared with a concurrent call
+ *   stream   cudaStream_t; the call enqueues a memset and three kernels
+ * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch; CUDA on
+ * launch failure.
+ */
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                       int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_kind,
+                       int window_l, int window_r, int draft_block, const int32_t* doc_ids,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * attn_decode_num_splits — how many KV splits attn_decode_splitkv uses.
  *
  * The keys [0, Lk_max) are cut into nsplit chunks of `chunk` keys each, a

@@ -25,7 +25,7 @@ __all__ = [
     "AttnError", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
-    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_decode_splitkv",
+    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_bwd", "attn_decode_splitkv",
     "attn_decode_num_splits", "SCORE_MOD_NONE", "SCORE_MOD_ALIBI",
     "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
@@ -47,8 +47,8 @@ SCORE_MOD_ALIBI = 1
 _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 
 EXPORTED_SYMBOLS = (
-    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_decode_num_splits",
-    "attn_decode_workspace_size",
+    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_bwd_workspace_size", "attn_bwd",
+    "attn_decode_num_splits", "attn_decode_workspace_size",
     "attn_decode_splitkv", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
 )
@@ -86,6 +86,11 @@ def load_library():
         lib.attn_fwd_score_mod.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
                                            i32, i32, i32, P, i32, P, P]
         lib.attn_fwd_score_mod.restype = i32
+        lib.attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
+        lib.attn_bwd_workspace_size.restype = sz
+        lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
+                                 i32, i32, i32, P, P, sz, P]
+        lib.attn_bwd.restype = i32
         lib.attn_fwd_varlen.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32,
                                         i32, i32, i32, i32, P]
         lib.attn_fwd_varlen.restype = i32
@@ -193,6 +198,42 @@ def attn_fwd_score_mod(q, k, v, *, alibi_slopes, scale=None, mask="none", window
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_score_mod")
     return o, lse
+
+
+def attn_bwd(q, k, v, o, lse, dout, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
+             doc_ids=None, workspace=None, dq=None, dk=None, dv=None, stream=None):
+    """Gradients of attn_fwd (see ``attn_bwd`` in include/attn.h): returns (dq, dk, dv).
+
+    q, o, dout: [B, Hq, Lq, d]; k, v: [B, Hkv, Lk, d] bf16 CUDA tensors; lse: fp32
+    [B, Hq, Lq] from attn_fwd with the same arguments.
+    """
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_bf16(name, t)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 CUDA tensor [B, Hq, Lq]")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    lib = load_library()
+    need = lib.attn_bwd_workspace_size(B, Hq, Lq, d)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if doc_ids is not None:
+        if doc_ids.dtype != torch.int32 or not doc_ids.is_cuda or not doc_ids.is_contiguous():
+            raise ValueError("doc_ids must be a contiguous int32 CUDA tensor [B, Lk]")
+    mk = mask if isinstance(mask, int) else _MASKS[mask]
+    st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                      _ptr(dk), _ptr(dv), B, Hq, Hkv, Lq, Lk, d, float(scale), mk, int(window[0]),
+                      int(window[1]), int(draft_block), _ptr(doc_ids), _ptr(workspace),
+                      workspace.numel() * workspace.element_size(),
+                      _stream_handle(stream, q.device))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, *, scale=None,

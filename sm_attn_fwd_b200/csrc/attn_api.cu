@@ -23,6 +23,9 @@ template <int D>
 cudaError_t launch_prefill(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                            const FwdParams&, int, cudaStream_t);
 int* device_error_word();
+template <int D>
+cudaError_t launch_backward(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                            const CUtensorMap&, const BwdParams&, cudaStream_t);
 cudaError_t launch_selftest_wait(cudaStream_t stream);
 }  // namespace attn
 
@@ -297,6 +300,76 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = d == 64 ? attn::launch_prefill<64>(tq, tk, tv, p, grid, st)
                           : attn::launch_prefill<128>(tq, tk, tv, p, grid, st);
+  return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Lq, int d) {
+  if (B < 1 || Hq < 1 || Lq < 1 || d < 1) return 0;
+  const size_t rows = (size_t)B * (size_t)Hq * (size_t)Lq;
+  const size_t acc = (rows * (size_t)d * 4 + 255) / 256 * 256;
+  return acc + rows * 4;
+}
+
+attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                       const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                       int Hq, int Hkv, int Lq, int Lk, int d, float scale, int mask_kind,
+                       int window_l, int window_r, int draft_block, const int32_t* doc_ids,
+                       void* workspace, size_t ws_bytes, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace)
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4) || !aligned(workspace, 256))
+    return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_DRAFT_BLOCK) return ATTN_ERR_INVALID_ARG;
+  if (window_l < -1 || window_r < -1) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_DRAFT_BLOCK && draft_block < 1) return ATTN_ERR_INVALID_ARG;
+  if (doc_ids && (!aligned(doc_ids, 4) || Lq > Lk)) return ATTN_ERR_INVALID_ARG;
+  if (d != 64) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)B * Hkv > kMaxGridY) return ATTN_ERR_UNSUPPORTED;
+  const size_t need = attn_bwd_workspace_size(B, Hq, Lq, d);
+  if (need == 0 || ws_bytes < need) return ATTN_ERR_WORKSPACE;
+
+  attn::BwdParams p;
+  std::memset(&p, 0, sizeof p);
+  p.o = o;
+  p.lse = lse;
+  p.dout = dout;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  const size_t rows = (size_t)B * Hq * Lq;
+  p.dq_acc = static_cast<float*>(workspace);
+  p.dsum = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                    (rows * (size_t)d * 4 + 255) / 256 * 256);
+  p.doc_ids = doc_ids;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.group = Hq / Hkv;
+  p.mask_kind = mask_kind;
+  p.window_l = window_l;
+  p.window_r = window_r;
+  p.draft_block = mask_kind == ATTN_MASK_DRAFT_BLOCK ? draft_block : 1;
+  p.scale = scale;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
+  p.q_tiles = (int)ceil_div(Lq, kBlockM);
+  p.err = error_word_for_current_device();
+  if (!p.err) return ATTN_ERR_CUDA;
+
+  CUtensorMap tq, tk, tv, tdo;
+  const uint64_t dq3[3] = {(uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq};
+  const uint64_t dk3[3] = {(uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv};
+  if (!encode_bf16(&tq, q, 3, dq3) || !encode_bf16(&tk, k, 3, dk3) ||
+      !encode_bf16(&tv, v, 3, dk3) || !encode_bf16(&tdo, dout, 3, dq3))
+    return ATTN_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(p.dq_acc, 0, rows * (size_t)d * 4, st) != cudaSuccess) return ATTN_ERR_CUDA;
+  cudaError_t e = attn::launch_backward<64>(tq, tk, tv, tdo, p, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -1,0 +1,457 @@
+// Backward pass of the attention forward for sm_100a (B200): dQ, dK, dV.
+//
+// Method ("FlashAttention 2 原理与 PyTorch 实战", section 3.2: the forward keeps
+// only O and the row statistics; the backward recomputes the scores tile by
+// tile instead of storing the N x N matrix).  With P the masked softmax of
+// S = scale * Q K^T:
+//   dV = P^T dO,  dP = dO V^T,  D_i = sum_c dO_ic O_ic,  dS = P * (dP - D),
+//   dQ = scale * dS K,  dK = scale * dS^T Q,
+// and P_ij = exp(S_ij - LSE_i) from the forward's log-sum-exp.
+//
+// B200 mapping.  One CTA per (b, kv head, 128-key tile), 192 threads; it keeps
+// its K and V tiles in shared memory and walks every query tile of every query
+// head of its group:
+//   warp 0     TMA producer: K and V once; per query tile Q, dO and, by all
+//              lanes, the tile's row statistics (LSE in base 2, D, document ids).
+//   warp 1     tcgen05.mma issue (elect.sync): S^T = K Q^T and dP^T = V dO^T
+//              (both operands K-major in shared memory), then dV += P^T dO and
+//              dK += dS^T Q (P^T, dS^T from tensor memory, dO, Q MN-major), and
+//              dQ_tile = dS K (dS from shared memory, MN-major, K MN-major).
+//   warps 2-5  one key per thread (its TMEM lane): P^T and dS^T for 128 query
+//              columns, written to tensor memory (bf16, over S^T and dP^T) and
+//              dS^T to shared memory; then, one query per thread, the dQ tile
+//              is reduced into an fp32 accumulator in global memory; at the end
+//              dK (times scale) and dV are stored as bf16.
+// Tensor memory (512 columns, d = 64): S^T / P^T [0,128), dP^T / dS^T
+// [128,256), dV [256,320), dK [320,384), dQ tile [384,448).
+// Small kernels before and after: D_i, and dQ from its fp32 accumulator.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "attn_params.h"
+#include "ptx.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kBwdThreads = 192;
+constexpr int kBwdTmemCols = 512;
+constexpr float kLog2eB = 1.44269504088896340736f;
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kAtomBytes = 128 * 128;       // one 64-column atom of a 128-row tile
+  static constexpr int kTileBytes = 128 * D * 2;     // one Q, K, V or dO tile
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;
+  static constexpr int kOffDO = kOffQ + kTileBytes;
+  static constexpr int kOffDS = kOffDO + kTileBytes;  // dS^T: [128 keys][128 queries] bf16
+  static constexpr int kOffStat = kOffDS + 2 * kAtomBytes;
+  static constexpr int kOffBar = kOffStat + 3 * 128 * 4;  // lse2, dsum, qdoc
+  static constexpr int kNumBars = 8;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  // tensor-memory columns
+  static constexpr uint32_t kST = 0, kDPT = 128, kDV = 256, kDK = 256 + D, kDQ = 256 + 2 * D;
+};
+
+enum : int { kBarKv = 0, kBarQFull, kBarQEmpty, kBarSFull, kBarPFull, kBarDqFull, kBarDqFree,
+             kBarAcc };
+
+__device__ __forceinline__ uint64_t bdesc(uint32_t addr, uint32_t lbo_bytes) {
+  return ptx::smem_desc_sw128(addr, lbo_bytes, 1024);
+}
+
+// Query positions [qlo, qhi] that key j may be seen from, before the document
+// test (every mask kind here gives an interval); hi < lo means none.
+__device__ __forceinline__ void query_bounds(const BwdParams& p, int j, int& qlo, int& qhi) {
+  const int off = p.Lk - p.Lq;  // query row i sits at position off + i
+  long long lo = 0, hi = (long long)p.Lq - 1;
+  if (p.mask_kind == kMaskCausal) {
+    lo = max(lo, (long long)j - off);
+  } else if (p.mask_kind == kMaskDraftBlock) {
+    const long long bd = p.draft_block;
+    lo = max(lo, (long long)(j / bd) * bd - off);
+  }
+  if (p.window_r >= 0) lo = max(lo, (long long)j - p.window_r - off);
+  if (p.window_l >= 0) hi = min(hi, (long long)j + p.window_l - off);
+  qlo = (int)max(-1LL, min(lo, (long long)p.Lq));
+  qhi = (int)max(-2LL, min(hi, (long long)p.Lq - 1));
+}
+
+// Does the key tile [k0, k0+127] meet the query tile [q0, q0+127]?  (Before the
+// document test, so a true answer may still have no visible pair.)
+__device__ __forceinline__ bool pair_live(const BwdParams& p, int k0, int q0) {
+  const int k_last = min(k0 + 127, p.Lk - 1);
+  int lo_a, hi_a, lo_b, hi_b;
+  query_bounds(p, k0, lo_a, hi_a);
+  query_bounds(p, k_last, lo_b, hi_b);
+  // the lower and upper bounds grow with the key index
+  return !(lo_a > q0 + 127 || hi_b < q0 || lo_a > hi_b);
+}
+
+// dQ_tile = dS K over 128 keys: 8 MMAs, A = dS in shared memory (MN-major,
+// 2048 bytes per 16 keys), B = K in shared memory (MN-major, same step).
+__device__ __forceinline__ void mma_ss_chain8_mn(uint32_t d_tmem, uint64_t a_desc,
+                                                 uint64_t b_desc, uint32_t idesc) {
+  for (int kk = 0; kk < 8; ++kk)
+    ptx::mma_ss_warp(d_tmem, a_desc + (uint64_t)(kk * 128), b_desc + (uint64_t)(kk * 128), idesc,
+                     kk > 0 ? 1u : 0u);
+}
+
+}  // namespace
+
+// D_i = sum_c dO_ic O_ic, one warp per query row.
+template <int D>
+__global__ void attn_bwd_dsum_kernel(const BwdParams p) {
+  const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long nrows = (long long)p.B * p.Hq * p.Lq;
+  if (row >= nrows) return;
+  const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(p.o) + row * D;
+  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(p.dout) + row * D;
+  float acc = 0.0f;
+#pragma unroll
+  for (int c = lane; c < D; c += 32) acc += __bfloat162float(o[c]) * __bfloat162float(g[c]);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) p.dsum[row] = acc;
+}
+
+// dQ (bf16) from its fp32 accumulator.
+__global__ void attn_bwd_dq_kernel(const BwdParams p, long long n) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) reinterpret_cast<__nv_bfloat16*>(p.dq)[i] = __float2bfloat16_rn(p.dq_acc[i]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using C = BwdCfg<D>;
+  static_assert(D == 64, "tensor memory holds S^T, dP^T, dV, dK and a dQ tile for d = 64");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sk = ptx::smem_u32(smem + C::kOffK);
+  const uint32_t sv = ptx::smem_u32(smem + C::kOffV);
+  const uint32_t sq = ptx::smem_u32(smem + C::kOffQ);
+  const uint32_t sdo = ptx::smem_u32(smem + C::kOffDO);
+  const uint32_t sds = ptx::smem_u32(smem + C::kOffDS);
+  float* lse2_s = reinterpret_cast<float*>(smem + C::kOffStat);
+  float* dsum_s = lse2_s + 128;
+  int* qdoc_s = reinterpret_cast<int*>(dsum_s + 128);
+  const uint32_t bar0 = ptx::smem_u32(smem + C::kOffBar);
+  auto BAR = [bar0](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  int* err = p.err;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int k0 = blockIdx.x * 128;
+  const int b = blockIdx.y / p.Hkv;
+  const int hkv = blockIdx.y % p.Hkv;
+  const int n_iter = p.group * p.q_tiles;  // (query head of the group, query tile)
+
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+    ptx::prefetch_tmap(&tm_do);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    ptx::mbar_init(&bars[kBarKv], 1);
+    ptx::mbar_init(&bars[kBarQFull], 1);
+    ptx::mbar_init(&bars[kBarQEmpty], 1);
+    ptx::mbar_init(&bars[kBarSFull], 1);
+    ptx::mbar_init(&bars[kBarPFull], 128);
+    ptx::mbar_init(&bars[kBarDqFull], 1);
+    ptx::mbar_init(&bars[kBarDqFree], 128);
+    ptx::mbar_init(&bars[kBarAcc], 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kBwdTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // the live (query head, query tile) pairs of this key tile, in order
+  auto iter_q0 = [&](int it) { return (it % p.q_tiles) * 128; };
+  auto iter_hq = [&](int it) { return hkv * p.group + it / p.q_tiles; };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    bool ok = true;
+    constexpr uint32_t kTx = C::kTileBytes;
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx_a(BAR(kBarKv), 2 * kTx);
+      for (int a = 0; a < D / 64; ++a) {
+        ptx::tma_load_3d_a(sk + a * C::kAtomBytes, &tm_k, BAR(kBarKv), a * 64, k0, b * p.Hkv + hkv);
+        ptx::tma_load_3d_a(sv + a * C::kAtomBytes, &tm_v, BAR(kBarKv), a * 64, k0, b * p.Hkv + hkv);
+      }
+    }
+    int n = 0;  // live pairs so far
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int q0 = iter_q0(it);
+      if (!pair_live(p, k0, q0)) continue;
+      const int hq = iter_hq(it);
+      const long long bh = (long long)b * p.Hq + hq;
+      if (n > 0) {
+        ok = ptx::mbar_wait_a(BAR(kBarQEmpty), (uint32_t)(n - 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutProducer);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      // row statistics of the query tile: LSE in base 2 (+inf for rows past Lq
+      // or with no visible key, so their P is 0), D, and the rows' documents
+      for (int r = lane; r < 128; r += 32) {
+        const int qi = q0 + r;
+        float l2 = INFINITY, dd = 0.0f;
+        int qd = 0;
+        if (qi < p.Lq) {
+          const float lse = __ldg(p.lse + bh * p.Lq + qi);
+          l2 = (lse == -INFINITY) ? INFINITY : lse * kLog2eB;
+          dd = __ldg(p.dsum + bh * p.Lq + qi);
+          if (p.doc_ids != nullptr) qd = __ldg(p.doc_ids + (long long)b * p.Lk + (p.Lk - p.Lq + qi));
+        }
+        lse2_s[r] = l2;
+        dsum_s[r] = dd;
+        qdoc_s[r] = qd;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx_a(BAR(kBarQFull), 2 * kTx);
+        for (int a = 0; a < D / 64; ++a) {
+          ptx::tma_load_3d_a(sq + a * C::kAtomBytes, &tm_q, BAR(kBarQFull), a * 64, q0, (int)bh);
+          ptx::tma_load_3d_a(sdo + a * C::kAtomBytes, &tm_do, BAR(kBarQFull), a * 64, q0, (int)bh);
+        }
+      }
+      ++n;
+    }
+    // drain: the last loads land before the CTA exits
+    if (lane == 0) {
+      int dummy = 0;
+      ptx::mbar_wait_a(BAR(kBarKv), 0, &dummy, nullptr, 0);
+      if (n > 0) {
+        dummy = 0;
+        ptx::mbar_wait_a(BAR(kBarQFull), (uint32_t)(n - 1) & 1u, &dummy, nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issue
+    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, 0, 0);   // K-major A and B
+    constexpr uint32_t kIdAcc = ptx::idesc_bf16_f32(128, D, 0, 1);   // A from TMEM, B MN-major
+    constexpr uint32_t kIdDq = ptx::idesc_bf16_f32(128, D, 1, 1);    // A and B MN-major
+    bool ok = ptx::mbar_wait_a(BAR(kBarKv), 0, abort_flag, err, kDevErrTimeoutMma);
+    ok = __all_sync(0xffffffffu, ok);
+    int n = 0;
+    for (int it = 0; it < n_iter && ok; ++it) {
+      if (!pair_live(p, k0, iter_q0(it))) continue;
+      ok = ptx::mbar_wait_a(BAR(kBarQFull), (uint32_t)n & 1u, abort_flag, err, kDevErrTimeoutMma);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      // S^T = K Q^T and dP^T = V dO^T (d = 64: one swizzle atom, 4 MMAs each)
+      ptx::mma_qk_chain_d64(tmem + C::kST, bdesc(sk, 16), bdesc(sq, 16), kIdS);
+      ptx::mma_qk_chain_d64(tmem + C::kDPT, bdesc(sv, 16), bdesc(sdo, 16), kIdS);
+      ptx::mma_commit_warp(BAR(kBarSFull));
+      // P^T, dS^T written (tensor memory and shared memory)
+      ok = ptx::mbar_wait_a(BAR(kBarPFull), (uint32_t)n & 1u, abort_flag, err, kDevErrTimeoutMma);
+      if (ok && n > 0)  // the previous dQ tile has been read out
+        ok = ptx::mbar_wait_a(BAR(kBarDqFree), (uint32_t)(n - 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutMma);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const uint32_t acc = n > 0 ? 1u : 0u;
+      ptx::mma_pv_chain8(tmem + C::kDV, tmem + C::kST, bdesc(sdo, C::kAtomBytes), kIdAcc, acc);
+      ptx::mma_pv_chain8(tmem + C::kDK, tmem + C::kDPT, bdesc(sq, C::kAtomBytes), kIdAcc, acc);
+      mma_ss_chain8_mn(tmem + C::kDQ, bdesc(sds, C::kAtomBytes), bdesc(sk, C::kAtomBytes), kIdDq);
+      ptx::mma_commit_warp(BAR(kBarQEmpty));
+      ptx::mma_commit_warp(BAR(kBarDqFull));
+      ++n;
+    }
+    ptx::mma_commit_warp(BAR(kBarAcc));
+  } else {
+    // ------------------------------------------------ P^T, dS^T and outputs
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;      // key of the tile (S^T lanes); query for dQ
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int key = k0 + row;
+    int qlo = 0, qhi = -1;
+    if (key < p.Lk) query_bounds(p, key, qlo, qhi);
+    const int kdoc = (p.doc_ids != nullptr && key < p.Lk)
+                         ? __ldg(p.doc_ids + (long long)b * p.Lk + key) : 0;
+    const float c = p.scale_log2;
+    bool ok = true;
+    int n = 0;
+    for (int it = 0; it < n_iter && ok; ++it) {
+      const int q0 = iter_q0(it);
+      if (!pair_live(p, k0, q0)) continue;
+      const int hq = iter_hq(it);
+      ok = ptx::mbar_wait_a(BAR(kBarSFull), (uint32_t)n & 1u, abort_flag, err,
+                            kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {  // 32 query columns at a time
+        uint32_t rs[32], rd[32];
+        ptx::tmem_ld32(t_row + C::kST + cc * 32, rs);
+        ptx::tmem_ld32(t_row + C::kDPT + cc * 32, rd);
+        ptx::tmem_wait_ld();
+        uint32_t pp[16], dp[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float pv[2], dv[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int col = cc * 32 + i + h;
+            const int qi = q0 + col;
+            bool vis = qi >= qlo && qi <= qhi;
+            if (p.doc_ids != nullptr) vis = vis && (qdoc_s[col] == kdoc);
+            const float l2 = lse2_s[col];
+            const float pe = vis ? ptx::ex2(__uint_as_float(rs[i + h]) * c - l2) : 0.0f;
+            pv[h] = (l2 == INFINITY) ? 0.0f : pe;
+            dv[h] = pv[h] * (__uint_as_float(rd[i + h]) - dsum_s[col]);
+          }
+          pp[i / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
+          dp[i / 2] = ptx::pack_bf16x2(dv[0], dv[1]);
+        }
+        // P^T and dS^T over the columns already read (16 columns per 32 queries)
+        ptx::tmem_st16(t_row + C::kST + cc * 16, pp);
+        ptx::tmem_st16(t_row + C::kDPT + cc * 16, dp);
+        // dS^T into shared memory as the MN-major A operand of dQ = dS K:
+        // row = key, 64 queries per 128-byte row of a swizzle atom
+        const uint32_t atom = sds + (uint32_t)((cc >> 1) * C::kAtomBytes) + (uint32_t)row * 128u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t chunk = (uint32_t)((cc & 1) * 4 + j);
+          const uint32_t addr = atom + ((chunk ^ (uint32_t)(row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dp[4 * j]),
+                       "r"(dp[4 * j + 1]), "r"(dp[4 * j + 2]), "r"(dp[4 * j + 3])
+                       : "memory");
+        }
+      }
+      ptx::tmem_wait_st();
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_a(BAR(kBarPFull));
+      // dQ tile: TMEM lane = query of the tile; reduce scale * dQ into the accumulator
+      ok = ptx::mbar_wait_a(BAR(kBarDqFull), (uint32_t)n & 1u, abort_flag, err,
+                            kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const int qi = q0 + row;
+      float* dst = p.dq_acc + (((long long)b * p.Hq + hq) * p.Lq + qi) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        ptx::tmem_ld32(t_row + C::kDQ + cc * 32, r);
+        ptx::tmem_wait_ld();
+        if (qi < p.Lq) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + cc * 32 + i),
+                         "f"(__uint_as_float(r[i]) * p.scale),
+                         "f"(__uint_as_float(r[i + 1]) * p.scale),
+                         "f"(__uint_as_float(r[i + 2]) * p.scale),
+                         "f"(__uint_as_float(r[i + 3]) * p.scale)
+                         : "memory");
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_a(BAR(kBarDqFree));
+      ++n;
+    }
+    // dK (times scale) and dV of this key tile
+    if (ok) {
+      ok = ptx::mbar_wait_a(BAR(kBarAcc), 0, abort_flag, err, kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    ptx::tc_fence_after();
+    if (key < p.Lk) {
+      const long long base = (((long long)b * p.Hkv + hkv) * p.Lk + key) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(which ? p.dv : p.dk) + base;
+        const float f = which ? 1.0f : p.scale;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          if (ok && n > 0) {
+            ptx::tmem_ld32(t_row + (which ? C::kDV : C::kDK) + cc * 32, r);
+            ptx::tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = 0u;
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            uint4 v4;
+            v4.x = ptx::pack_bf16x2(__uint_as_float(r[i]) * f, __uint_as_float(r[i + 1]) * f);
+            v4.y = ptx::pack_bf16x2(__uint_as_float(r[i + 2]) * f, __uint_as_float(r[i + 3]) * f);
+            v4.z = ptx::pack_bf16x2(__uint_as_float(r[i + 4]) * f, __uint_as_float(r[i + 5]) * f);
+            v4.w = ptx::pack_bf16x2(__uint_as_float(r[i + 6]) * f, __uint_as_float(r[i + 7]) * f);
+            *reinterpret_cast<uint4*>(out + cc * 32 + i) = v4;
+          }
+        }
+      }
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kBwdTmemCols);
+  }
+}
+
+// The three launches of the backward: D_i, the main kernel, dQ to bf16.  The
+// caller zeroes dq_acc before (on the same stream).
+template <int D>
+cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+  const long long nrows = (long long)p.B * p.Hq * p.Lq;
+  attn_bwd_dsum_kernel<D><<<(unsigned)((nrows + 7) / 8), 256, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto kern = attn_bwd_kernel<D>;
+  constexpr int smem = BwdCfg<D>::kSmemAlloc;
+  static bool configured[64] = {};
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  const dim3 grid((unsigned)((p.Lk + 127) / 128), (unsigned)(p.B * p.Hkv), 1);
+  kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n = nrows * D;
+  attn_bwd_dq_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p, n);
+  return cudaGetLastError();
+}
+
+template cudaError_t launch_backward<64>(const CUtensorMap&, const CUtensorMap&,
+                                         const CUtensorMap&, const CUtensorMap&,
+                                         const BwdParams&, cudaStream_t);
+
+}  // namespace attn

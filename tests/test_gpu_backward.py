@@ -1,0 +1,66 @@
+"""GPU parity of attn_bwd (dQ, dK, dV) against the double-precision backward oracle.
+
+Tolerance: the kernel rounds P and dS to bf16 before the MMAs and writes bf16
+gradients, so each gradient is compared against the oracle's with
+max |d| <= 3e-2 * max|ref| and mean |d| <= 3e-3 * max|ref| (per tensor)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sm_attn_fwd_b200 as ab
+from tests.gpu_helpers import to_dev
+from workloads import random_case
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(got, ref, what):
+    g = got.float().cpu().double().numpy()
+    scale = max(1e-6, np.abs(ref).max())
+    err = np.abs(g - ref)
+    assert np.isfinite(g).all(), what
+    assert err.max() <= 3e-2 * scale and err.mean() <= 3e-3 * scale, \
+        f"{what}: max {err.max():.3g} mean {err.mean():.3g} ref max {scale:.3g}"
+
+
+CASES = [
+    # seed, B, Hq, Hkv, Lq, Lk, mask, window, bd, doc
+    (1, 1, 2, 2, 128, 128, "none", (-1, -1), 1, False),
+    (2, 1, 2, 2, 256, 256, "causal", (-1, -1), 1, False),
+    (3, 2, 4, 2, 200, 333, "causal", (-1, -1), 1, False),
+    (4, 1, 2, 1, 300, 300, "none", (40, 17), 1, True),
+    (5, 1, 2, 2, 160, 400, "draft", (-1, 64), 16, False),
+    (6, 1, 8, 2, 129, 129, "causal", (50, 0), 1, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"s{c[0]}_{c[6]}_lq{c[4]}_lk{c[5]}")
+def test_backward_matches_oracle(case):
+    seed, B, Hq, Hkv, Lq, Lk, mask, window, bd, doc = case
+    d = 64
+    q, k, v, doc_ids, _ = random_case(seed, B, Hq, Hkv, Lq, Lk, d, doc_split=doc, n_docs=3)
+    do = torch.randn(B, Hq, Lq, d, generator=torch.Generator().manual_seed(seed + 100))
+    do = do.to(torch.bfloat16)
+    kw = dict(scale=1.0 / math.sqrt(d), mask=mask, window=window, draft_block=bd)
+    qd, kd, vd, dod = to_dev(q, k, v, do)
+    docd = None if doc_ids is None else doc_ids.cuda()
+    o, lse = ab.attn_fwd(qd, kd, vd, doc_ids=docd, **kw)
+    dq, dk, dv = ab.attn_bwd(qd, kd, vd, o, lse, dod, doc_ids=docd, **kw)
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    rq, rk, rv = oracle.attn_bwd(q, k, v, do, doc_ids=doc_ids, **kw)
+    _check(dv, rv, f"dV {case}")
+    _check(dk, rk, f"dK {case}")
+    _check(dq, rq, f"dQ {case}")
+
+
+def test_backward_rejects_on_host():
+    q = torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros(1, 2, 64, dtype=torch.float32, device="cuda")
+    with pytest.raises(ab.AttnError) as e:
+        ab.attn_bwd(q, q, q, q, lse, q)               # d = 128 not built
+    assert e.value.status == ab.ATTN_ERR_UNSUPPORTED

@@ -55,7 +55,8 @@ struct BwdCfg {
   static constexpr int kNumBars = 8;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
-  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  // at least 120 KB, so one CTA per SM holds the whole tensor memory
+  static constexpr int kSmemAlloc = (kSmemBytes + 1024 > 120 * 1024) ? kSmemBytes + 1024 : 120 * 1024;
   // tensor-memory columns
   static constexpr uint32_t kST = 0, kDPT = 128, kDV = 256, kDK = 256 + D, kDQ = 256 + 2 * D;
 };
@@ -381,22 +382,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = __all_sync(0xffffffffu, ok);
     }
     ptx::tc_fence_after();
-    if (key < p.Lk) {
-      const long long base = (((long long)b * p.Hkv + hkv) * p.Lk + key) * D;
+    // tcgen05.ld is warp-collective: every lane loads, only keys below Lk store
+    const long long base = (((long long)b * p.Hkv + hkv) * p.Lk + key) * D;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(which ? p.dv : p.dk) + base;
-        const float f = which ? 1.0f : p.scale;
+    for (int which = 0; which < 2; ++which) {
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(which ? p.dv : p.dk) + base;
+      const float f = which ? 1.0f : p.scale;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t r[32];
-          if (ok && n > 0) {
-            ptx::tmem_ld32(t_row + (which ? C::kDV : C::kDK) + cc * 32, r);
-            ptx::tmem_wait_ld();
-          } else {
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        if (ok && n > 0) {  // warp-uniform
+          ptx::tmem_ld32(t_row + (which ? C::kDV : C::kDK) + cc * 32, r);
+          ptx::tmem_wait_ld();
+        } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = 0u;
-          }
+          for (int i = 0; i < 32; ++i) r[i] = 0u;
+        }
+        if (key < p.Lk) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
             uint4 v4;

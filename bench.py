@@ -247,6 +247,30 @@ def run_alibi(cfg, timer, steps, warmup, stream):
     return ms, algorithmic_flops(cfg, visible_pairs(cfg))
 
 
+def run_backward(cfg, timer, steps, warmup, stream):
+    """attn_bwd on a prefill workload (d = 64).  Work: the two score GEMMs and three
+    gradient GEMMs of 2*d flop per visible pair each, 10*d*pairs in all."""
+    import sm_attn_fwd_b200 as ab
+    inp = make_inputs(cfg, device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(cfg.seed + 1000)
+    dout = torch.randn(inp.q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    torch.cuda.synchronize()
+    o, lse = ab.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask,
+                         stream=stream)
+    ws = torch.empty(ab.load_library().attn_bwd_workspace_size(cfg.B, cfg.Hq, cfg.Lq, cfg.d),
+                     dtype=torch.uint8, device="cuda")
+    dq, dk, dv = torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v)
+    fn = lambda: ab.attn_bwd(inp.q, inp.k, inp.v, o, lse, dout, scale=cfg.softmax_scale,  # noqa: E731
+                             mask=cfg.mask, workspace=ws, dq=dq, dk=dk, dv=dv, stream=stream)
+    ms = timer.time(fn, steps, warmup)
+    st, bits = ab.attn_get_device_error(stream)
+    if st != ab.ATTN_OK:
+        raise RuntimeError(f"device error after attn_bwd on {cfg.name}: {st} {bits}")
+    pairs = visible_pairs(cfg) * cfg.Hq
+    return ms, 10.0 * cfg.d * pairs
+
+
 # Packed sequences: 16 documents with lengths drawn uniformly from [128, 4096]
 # (seed 5), self-attention, causal, H = 16, d = 64.
 VARLEN_NAME = "varlen_causal_16seqs_l128to4096_h16_d64"
@@ -468,6 +492,8 @@ def main():
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: total CPU seconds across all steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time attn_bwd on the headline workload (reported under workloads)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" and args.only is None else args.warmup
 
@@ -521,6 +547,13 @@ def main():
                                                    "TFLOP/s": tf,
                                                    "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
                                                    "algorithmic_flop": fl6}
+            if args.backward:
+                ms7, fl7 = run_backward(HEADLINE, timer, max(5, args.steps // 10), 3, stream)
+                med = statistics.median(ms7)
+                tf = fl7 / (med * 1e9)
+                workloads[HEADLINE.name + "_backward"] = {
+                    "ms_median": med, "ms_min": min(ms7), "TFLOP/s": tf,
+                    "frac_of_bf16_peak": tf / peaks["bf16_tflops"], "algorithmic_flop": fl7}
             ms5, fl5, lens5 = run_varlen(timer, max(5, args.steps // 10), 3, stream)
             med = statistics.median(ms5)
             tf = fl5 / (med * 1e9)

@@ -149,3 +149,25 @@ def test_attn_fwd_score_mod_rejects_on_host():
     bad_d = list(args)
     bad_d[10] = 96
     assert lib.attn_fwd_score_mod(*bad_d) == ab.ATTN_ERR_UNSUPPORTED
+
+
+def test_attn_bwd_rejects_on_host_and_sizes_its_workspace():
+    lib = ab.load_library()
+    B, Hq, Hkv, Lq, Lk, d = 2, 8, 2, 100, 130, 64
+    need = lib.attn_bwd_workspace_size(B, Hq, Lq, d)
+    rows = B * Hq * Lq
+    assert need == (rows * d * 4 + 255) // 256 * 256 + rows * 4
+    assert lib.attn_bwd_workspace_size(0, Hq, Lq, d) == 0
+    #      q  k  v  o  lse dout dq dk dv
+    ptrs = [A, A, A, A, A, A, A, A, A]
+    tail = [B, Hq, Hkv, Lq, Lk, d, 0.125, 1, -1, -1, 1, None, A, need, None]
+    assert lib.attn_bwd(*ptrs[:8], None, *tail) == ab.ATTN_ERR_INVALID_ARG       # no dv
+    small = list(tail)
+    small[13] = need - 1
+    assert lib.attn_bwd(*ptrs, *small) == ab.ATTN_ERR_WORKSPACE
+    d128 = list(tail)
+    d128[5] = 128
+    assert lib.attn_bwd(*ptrs, *d128) == ab.ATTN_ERR_UNSUPPORTED
+    bad_ws = list(tail)
+    bad_ws[12] = ctypes.c_void_p(0x10010)                                       # not 256-aligned
+    assert lib.attn_bwd(*ptrs, *bad_ws) == ab.ATTN_ERR_INVALID_ARG

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "attn_bwd_params.h"
 #include "attn_params.h"
 
 namespace attn {

@@ -31,6 +31,7 @@
 
 #include <cstdint>
 
+#include "attn_bwd_params.h"
 #include "attn_params.h"
 #include "ptx.cuh"
 

@@ -11,7 +11,11 @@ two-pass softmax over each materialised score row ("FlashAttention 2 原理与
 PyTorch 实战", sections 一 and 3.2); ``mask`` is the mask_mod predicate
 ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", sections 1 and 3);
 ``decode_partials`` and ``combine`` are the split-KV decode written out as
-chunk-then-merge (same page, section 1).
+chunk-then-merge (same page, section 1); ``paged_gather`` reads a paged cache
+through its block table; ``attn_fwd_varlen`` applies the definition to each of
+a batch of packed sequences; ``alibi_slopes`` adds the ALiBi score_mod (same
+page, section 1); ``attn_bwd`` writes out the gradients dQ, dK, dV of the
+definition on whole score rows (numpy, double).
 """
 from __future__ import annotations
 

@@ -171,3 +171,20 @@ def test_attn_bwd_rejects_on_host_and_sizes_its_workspace():
     bad_ws = list(tail)
     bad_ws[12] = ctypes.c_void_p(0x10010)                                       # not 256-aligned
     assert lib.attn_bwd(*ptrs, *bad_ws) == ab.ATTN_ERR_INVALID_ARG
+
+
+def test_binding_checks_tensors_before_calling_the_library():
+    """The Python binding rejects host tensors, wrong dtypes and wrong ranks itself."""
+    import torch
+    q4 = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)          # host tensor
+    with pytest.raises(ValueError, match="CUDA"):
+        ab.attn_fwd(q4, q4, q4)
+    with pytest.raises(ValueError, match="CUDA"):
+        ab.attn_fwd_score_mod(q4, q4, q4, alibi_slopes=torch.zeros(2))
+    q3 = torch.zeros(8, 2, 64, dtype=torch.bfloat16)
+    cu = torch.tensor([0, 8], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        ab.attn_fwd_varlen(q3, q3, q3, cu, cu, 8)
+    lse = torch.zeros(1, 2, 8)
+    with pytest.raises(ValueError, match="CUDA"):
+        ab.attn_bwd(q4, q4, q4, q4, lse, q4)

@@ -60,39 +60,69 @@ def load_peaks():
                 "source": "fallback"}
 
 
-def visible_pairs(cfg, doc_ids=None, kv_lens=None) -> int:
-    """Visible (query, key) pairs of one head summed over the batch.
+def _row_intervals(cfg, b, doc_ids=None, kv_lens=None):
+    """Visible key interval [lo, hi] of every query row of sequence b.
 
-    Every mask here gives each query row one contiguous key interval
-    [lo, hi]; the document mask then keeps the keys of the row's document.
+    Every mask here gives each query row one contiguous key interval; the
+    document mask then keeps the keys of the row's document, which is again
+    an interval because documents are contiguous runs of positions.
     """
-    B, Lq, Lk = cfg.B, cfg.Lq, cfg.Lk
+    Lq, Lk = cfg.Lq, cfg.Lk
+    lkb = Lk if kv_lens is None else int(kv_lens[b])
+    p = np.arange(Lq, dtype=np.int64) + (lkb - Lq)
+    lo = np.zeros(Lq, dtype=np.int64)
+    hi = np.full(Lq, lkb - 1, dtype=np.int64)
+    if cfg.mask == "causal":
+        hi = np.minimum(hi, p)
+    elif cfg.mask == "draft":
+        bd = cfg.draft_block
+        hi = np.minimum(hi, (np.floor_divide(p, bd) + 1) * bd - 1)
+    wl, wr = cfg.window
+    if wl >= 0:
+        lo = np.maximum(lo, p - wl)
+    if wr >= 0:
+        hi = np.minimum(hi, p + wr)
+    if doc_ids is not None:
+        d = np.asarray(doc_ids[b], dtype=np.int64)
+        starts = np.concatenate([[0], np.nonzero(np.diff(d))[0] + 1])
+        ends = np.concatenate([starts[1:], [Lk]]) - 1
+        run = np.searchsorted(starts, p, side="right") - 1
+        lo = np.maximum(lo, starts[run])
+        hi = np.minimum(hi, ends[run])
+    return lo, hi
+
+
+def visible_pairs(cfg, doc_ids=None, kv_lens=None) -> int:
+    """Visible (query, key) pairs of one head summed over the batch."""
     total = 0
-    for b in range(B):
-        lkb = Lk if kv_lens is None else int(kv_lens[b])
-        p = np.arange(Lq, dtype=np.int64) + (lkb - Lq)
-        lo = np.zeros(Lq, dtype=np.int64)
-        hi = np.full(Lq, lkb - 1, dtype=np.int64)
-        if cfg.mask == "causal":
-            hi = np.minimum(hi, p)
-        elif cfg.mask == "draft":
-            bd = cfg.draft_block
-            hi = np.minimum(hi, (np.floor_divide(p, bd) + 1) * bd - 1)
-        wl, wr = cfg.window
-        if wl >= 0:
-            lo = np.maximum(lo, p - wl)
-        if wr >= 0:
-            hi = np.minimum(hi, p + wr)
-        if doc_ids is not None:
-            d = np.asarray(doc_ids[b], dtype=np.int64)
-            # documents are contiguous runs of positions: clip to the row's run
-            starts = np.concatenate([[0], np.nonzero(np.diff(d))[0] + 1])
-            ends = np.concatenate([starts[1:], [Lk]]) - 1
-            run = np.searchsorted(starts, p, side="right") - 1
-            lo = np.maximum(lo, starts[run])
-            hi = np.minimum(hi, ends[run])
+    for b in range(cfg.B):
+        lo, hi = _row_intervals(cfg, b, doc_ids, kv_lens)
         total += int(np.maximum(hi - lo + 1, 0).sum())
     return total
+
+
+def visible_keys(cfg, doc_ids=None) -> int:
+    """Keys that at least one query row sees, summed over the batch (one head)."""
+    total = 0
+    for b in range(cfg.B):
+        lo, hi = _row_intervals(cfg, b, doc_ids)
+        seen = np.zeros(cfg.Lk + 1, dtype=np.int64)
+        ok = hi >= lo
+        np.add.at(seen, lo[ok], 1)
+        np.add.at(seen, hi[ok] + 1, -1)
+        total += int((np.cumsum(seen)[: cfg.Lk] > 0).sum())
+    return total
+
+
+def prefill_bytes(cfg, doc_ids=None) -> float:
+    """Algorithmic HBM bytes of one prefill call: Q read, the K and V rows some
+    query row sees (every KV head), O written, LSE written (and the document
+    ids of the batch when given)."""
+    q = cfg.B * cfg.Hq * cfg.Lq * cfg.d * 2
+    kv = visible_keys(cfg, doc_ids) * cfg.Hkv * cfg.d * 2 * 2
+    lse = cfg.B * cfg.Hq * cfg.Lq * 4
+    doc = 0 if doc_ids is None else cfg.B * cfg.Lk * 4
+    return float(2 * q + kv + lse + doc)
 
 
 def algorithmic_flops(cfg, pairs_per_head):
@@ -183,6 +213,18 @@ def profiled_traffic():
 
 
 # ----------------------------------------------------------- GPU timing
+def device_inputs(cfg):
+    """The workload's inputs drawn with the CPU generator (the same draws the
+    parity tests check against the oracle), then copied to the GPU."""
+    inp = make_inputs(cfg, device="cpu")
+    for name in ("q", "k", "v", "doc_ids", "kv_lens"):
+        t = getattr(inp, name)
+        if t is not None:
+            setattr(inp, name, t.to("cuda").contiguous())
+    torch.cuda.synchronize()
+    return inp
+
+
 class Timer:
     """CUDA-event timing of single launches on one stream, L2 flushed before each."""
 
@@ -212,8 +254,7 @@ class Timer:
 def run_prefill(cfg, timer, steps, warmup, stream, batch_mult=1):
     import sm_attn_fwd_b200 as ab
     c = cfg.with_(B=cfg.B * batch_mult) if batch_mult != 1 else cfg
-    inp = make_inputs(c, device="cuda")
-    torch.cuda.synchronize()  # inputs are drawn on the default stream; launches use `stream`
+    inp = device_inputs(c)
     o = torch.empty_like(inp.q)
     lse = torch.empty(c.B, c.Hq, c.Lq, dtype=torch.float32, device="cuda")
     kw = dict(scale=c.softmax_scale, mask=c.mask, window=c.window, draft_block=c.draft_block,
@@ -225,13 +266,13 @@ def run_prefill(cfg, timer, steps, warmup, stream, batch_mult=1):
         raise RuntimeError(f"device error after {c.name}: {st} {bits}")
     doc = None if inp.doc_ids is None else inp.doc_ids.cpu().numpy()
     pairs = visible_pairs(c, doc_ids=doc)
-    return c, inp, ms, algorithmic_flops(c, pairs)
+    return c, inp, ms, algorithmic_flops(c, pairs), prefill_bytes(c, doc_ids=doc)
 
 
 def run_alibi(cfg, timer, steps, warmup, stream):
     """The headline workload with the ALiBi score_mod (slopes 2^(-8 (h+1) / H))."""
     import sm_attn_fwd_b200 as ab
-    inp = make_inputs(cfg, device="cuda")
+    inp = device_inputs(cfg)
     slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / cfg.Hq) for h in range(cfg.Hq)],
                           dtype=torch.float32, device="cuda")
     torch.cuda.synchronize()
@@ -251,10 +292,10 @@ def run_backward(cfg, timer, steps, warmup, stream):
     """attn_bwd on a prefill workload (d = 64).  Work: the two score GEMMs and three
     gradient GEMMs of 2*d flop per visible pair each, 10*d*pairs in all."""
     import sm_attn_fwd_b200 as ab
-    inp = make_inputs(cfg, device="cuda")
-    g = torch.Generator(device="cuda")
+    inp = device_inputs(cfg)
+    g = torch.Generator()
     g.manual_seed(cfg.seed + 1000)
-    dout = torch.randn(inp.q.shape, generator=g, device="cuda").to(torch.bfloat16)
+    dout = torch.randn(inp.q.shape, generator=g).to(torch.bfloat16).cuda()
     torch.cuda.synchronize()
     o, lse = ab.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask,
                          stream=stream)
@@ -280,7 +321,7 @@ def run_varlen(timer, steps, warmup, stream, *, n=16, lo=128, hi=4096, H=16, d=6
     import sm_attn_fwd_b200 as ab
     from workloads import packed_case, packed_lengths
     lens = packed_lengths(seed, n, lo, hi)
-    q, k, v, cu_q, cu_k = packed_case(seed, lens, lens, H, H, d, device="cuda")
+    q, k, v, cu_q, cu_k = (t.cuda() for t in packed_case(seed, lens, lens, H, H, d))
     torch.cuda.synchronize()
     o = torch.empty_like(q)
     lse = torch.empty(H, q.shape[0], dtype=torch.float32, device="cuda")
@@ -521,8 +562,8 @@ def main():
             _, ms, nbytes, plan = run_decode(cfg, timer, args.steps, args.warmup, stream)
             print(json.dumps({"workload": cfg.name, "ms": ms, "GB/s": nbytes / (statistics.median(ms) * 1e6)}))
         else:
-            c, _, ms, flops = run_prefill(cfg, timer, args.steps, args.warmup, stream,
-                                          batch_mult=args.batch_mult)
+            c, _, ms, flops, _ = run_prefill(cfg, timer, args.steps, args.warmup, stream,
+                                             batch_mult=args.batch_mult)
             print(json.dumps({"workload": c.name, "ms": ms,
                               "TFLOP/s": flops / (statistics.median(ms) * 1e9)}))
         return
@@ -530,16 +571,19 @@ def main():
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
-        cfg, _, ms, flops = run_prefill(HEADLINE, timer, args.steps, args.warmup, stream)
+        cfg, _, ms, flops, _ = run_prefill(HEADLINE, timer, args.steps, args.warmup, stream)
         workloads = {}
         if not args.no_secondary:
             for sc in (CAUSAL_32K_GQA, DRAFT_WINDOW_DOC, DRAFT_WINDOW_DOC_FULL):
-                c2, _, ms2, fl2 = run_prefill(sc, timer, max(3, args.steps // 20), 3, stream)
+                c2, _, ms2, fl2, by2 = run_prefill(sc, timer, max(3, args.steps // 20), 3, stream)
                 med = statistics.median(ms2)
                 tf = fl2 / (med * 1e9)
+                gbs = by2 / (med * 1e6)
                 workloads[c2.name] = {"ms_median": med, "ms_min": min(ms2), "TFLOP/s": tf,
                                       "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
-                                      "algorithmic_flop": fl2}
+                                      "algorithmic_flop": fl2, "GB/s": gbs,
+                                      "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                                      "algorithmic_bytes": by2}
             ms6, fl6 = run_alibi(HEADLINE, timer, max(5, args.steps // 10), 3, stream)
             med = statistics.median(ms6)
             tf = fl6 / (med * 1e9)

@@ -30,6 +30,13 @@
  *     read by attn_get_device_error().
  *   - Inputs must be finite, except the decode cache past kv_lens[b], which
  *     may hold anything (it is never used, not even multiplied by zero).
+ *   - The device error word is ONE word per device, shared by every stream,
+ *     every host thread and every entry point of the library: a bit set by
+ *     one caller's kernel is seen (and cleared) by whichever caller next
+ *     calls attn_get_device_error on that device.
+ *   - Per-device set-up (shared-memory opt-ins, symbol addresses) is done by
+ *     a device's first call in each CUDA context, so the library stays usable
+ *     after cudaDeviceReset; make that first call outside any stream capture.
  */
 #ifndef ATTN_B200_ATTN_H_
 #define ATTN_B200_ATTN_H_
@@ -182,6 +189,9 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Lq, int d);
  *   workspace  device memory, 256-byte aligned, >= attn_bwd_workspace_size bytes,
  *            owned by the caller, not shared with a concurrent call
  *   stream   cudaStream_t; the call enqueues a memset and three kernels
+ * Determinism: dK and dV are bit-identical from run to run; dQ is not, since
+ * its fp32 accumulator receives one atomic add per (key tile, query tile)
+ * pair in whatever order the CTAs run (differences are rounding-level).
  * Errors: INVALID_ARG / UNSUPPORTED / WORKSPACE before any launch; CUDA on
  * launch failure.
  */
@@ -294,7 +304,8 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
  *   - Every GPU that loads the library holds that array until the process
  *     exits.
  *   - The first call on a device looks up the array's device address (with
- *     that device current); make this first call before any stream capture.
+ *     that device current, and again in a new context after
+ *     cudaDeviceReset); make this first call before any stream capture.
  *   - Requests whose attn_decode_workspace_size(...) exceeds 32 MiB return
  *     ATTN_ERR_WORKSPACE and launch nothing (e.g. B=64, Hq=64, Lq=1,
  *     Lk_max=32768, d=128 needs 16.9 MB and fits; the Lq=16 variant does not).
@@ -313,7 +324,8 @@ attn_status_t attn_decode_splitkv_noalloc(const void* q, const void* k_cache,
 
 /*
  * attn_get_device_error — synchronise `stream`, then read and clear the
- * device error word of the current device.  Returns ATTN_OK, ATTN_ERR_TIMEOUT
+ * device error word of the current device (shared by all callers; see the
+ * conventions above).  Returns ATTN_OK, ATTN_ERR_TIMEOUT
  * (a kernel abandoned a bounded wait), ATTN_ERR_INVALID_ARG (a kv_lens entry
  * or a block_table page id was out of range) or ATTN_ERR_CUDA (the
  * synchronisation itself failed).

@@ -13,6 +13,7 @@
 #include "attn.h"
 #include "attn_bwd_params.h"
 #include "attn_params.h"
+#include "host_once.h"
 
 namespace attn {
 template <int D>
@@ -51,6 +52,34 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   });
   return fn;
 }
+
+}  // namespace
+
+unsigned long long attn::current_context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &qres) ==
+            cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(ptr);
+    ptr = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
+        qres == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(ptr);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -106,15 +135,22 @@ int num_sms() {
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 
-// Device address of the kernels' error word, looked up once per device.
+// Device address of the kernels' error word, looked up once per device and
+// context.
 int* error_word_for_current_device() {
-  static int* cache[64] = {};
-  static std::mutex mu;
+  static attn::PerContextOnce once;
+  static int* cache[attn::kMaxDevices] = {};
+  int* out = nullptr;
+  const cudaError_t e = attn::once_per_context(once, [&](int dev) {
+    cache[dev] = attn::device_error_word();
+    return cache[dev] ? cudaSuccess : cudaErrorInvalidSymbol;
+  });
+  if (e != cudaSuccess) return nullptr;
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!cache[dev]) cache[dev] = attn::device_error_word();
-  return cache[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  std::lock_guard<std::mutex> lock(once.mu);
+  out = cache[dev];
+  return out;
 }
 
 struct SplitPlan {

@@ -33,6 +33,7 @@
 
 #include "attn_bwd_params.h"
 #include "attn_params.h"
+#include "host_once.h"
 #include "ptx.cuh"
 
 namespace attn {
@@ -434,16 +435,11 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   if (e != cudaSuccess) return e;
   auto kern = attn_bwd_kernel<D>;
   constexpr int smem = BwdCfg<D>::kSmemAlloc;
-  static bool configured[64] = {};
-  int dev = 0;
-  e = cudaGetDevice(&dev);
+  static PerContextOnce once;
+  e = once_per_context(once, [&](int) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
   const dim3 grid((unsigned)((p.Lk + 127) / 128), (unsigned)(p.B * p.Hkv), 1);
   kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
   e = cudaGetLastError();

@@ -30,6 +30,7 @@
 #include <cstdint>
 
 #include "attn_params.h"
+#include "host_once.h"
 #include "ptx.cuh"
 
 namespace attn {
@@ -592,18 +593,13 @@ cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           const FwdParams& p, dim3 grid, cudaStream_t stream) {
   auto kern = attn_decode_kernel<D>;
   constexpr int smem = Cfg<D>::kSmemAlloc;
-  // The shared-memory opt-in is set once per device, outside any stream capture
-  // that a later call may be part of.
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  // The shared-memory opt-in is set once per device and context, normally by
+  // a first call outside any stream capture that a later call may be part of.
+  static PerContextOnce once;
+  const cudaError_t e = once_per_context(once, [&](int) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

@@ -15,6 +15,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "host_once.h"
 
 namespace {
 
@@ -24,24 +25,28 @@ constexpr size_t kNoAllocWorkspaceBytes = 32u << 20;  // 32 MiB
 // symbol, not a device address: the address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_workspace[kNoAllocWorkspaceBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_workspace_ptr[kMaxDevices] = {};
+attn::PerContextOnce g_setup;
+void* g_workspace_ptr[attn::kMaxDevices] = {};
 
-// Once per device, with that device current: the device address of the array.
+// Once per device (and again in a new context, e.g. after cudaDeviceReset),
+// with that device current: the device address of the array.
 attn_status_t workspace_for_current_device(void** out) {
+  const cudaError_t e = attn::once_per_context(g_setup, [](int dev) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_workspace) != cudaSuccess || ptr == nullptr) {
+      g_workspace_ptr[dev] = nullptr;
+      return cudaErrorInvalidSymbol;
+    }
+    g_workspace_ptr[dev] = ptr;
+    return cudaSuccess;
+  });
+  if (e == cudaErrorInvalidDevice) return ATTN_ERR_UNSUPPORTED;
+  if (e != cudaSuccess) return ATTN_ERR_CUDA;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_workspace_ptr[dev] == nullptr) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_workspace) != cudaSuccess || ptr == nullptr)
-      return ATTN_ERR_CUDA;
-    g_workspace_ptr[dev] = ptr;
-  }
+  std::lock_guard<std::mutex> lock(g_setup.mu);
   *out = g_workspace_ptr[dev];
-  return ATTN_OK;
+  return *out ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 }  // namespace

@@ -33,6 +33,7 @@
 #include <type_traits>
 
 #include "attn_params.h"
+#include "host_once.h"
 #include "ptx.cuh"
 
 namespace attn {
@@ -1062,16 +1063,11 @@ cudaError_t launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tk,
                                   cudaStream_t stream) {
   auto kern = attn_prefill_kernel<D, kAlibi>;
   constexpr int smem = Cfg<D>::kSmemAlloc;
-  static bool configured[64] = {};
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static PerContextOnce once;
+  const cudaError_t e = once_per_context(once, [&](int) {
+    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  });
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!configured[dev]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    configured[dev] = true;
-  }
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

@@ -109,29 +109,24 @@ def test_bad_kv_len_is_flagged_not_faulted():
 
 
 @pytest.mark.parametrize("cfg", [DECODE_LQ1, DECODE_LQ16], ids=lambda c: c.name)
-def test_config_decode_sampled(cfg):
-    """Full-size decode (inputs drawn on the GPU); sampled (b, kv head) groups
-    are checked against the oracle on their own slice of the cache."""
+def test_config_decode_full(cfg):
+    """Full-size decode, every sequence and every head.  The 8.6 GB cache is
+    drawn on the GPU with the workload recipe (the draws the bench times);
+    each sequence's first kv_lens[b] keys are copied back and checked against
+    the oracle."""
     inp = make_inputs(cfg, device="cuda")
     o, lse = ab.attn_decode_splitkv(inp.q, inp.k, inp.v, inp.kv_lens)
     torch.cuda.synchronize()
     st, bits = ab.attn_get_device_error()
     assert st == ab.ATTN_OK, (st, bits)
-    G = cfg.Hq // cfg.Hkv
-    rng = np.random.default_rng(5)
     kv_host = inp.kv_lens.cpu()
-    picks = {(0, 0), (cfg.B - 1, cfg.Hkv - 1), (int(torch.argmax(kv_host)), 3),
-             (int(torch.argmin(kv_host)), 5)}
-    while len(picks) < 10:
-        picks.add((int(rng.integers(cfg.B)), int(rng.integers(cfg.Hkv))))
-    for b, h in sorted(picks):
+    for b in range(cfg.B):
         L = int(kv_host[b])
-        qs = inp.q[b:b + 1, h * G:(h + 1) * G].cpu()
-        ks = inp.k[b:b + 1, h:h + 1, :L].cpu()
-        vs = inp.v[b:b + 1, h:h + 1, :L].cpu()
+        qs = inp.q[b:b + 1].cpu()
+        ks = inp.k[b:b + 1, :, :L].cpu()
+        vs = inp.v[b:b + 1, :, :L].cpu()
         ro, rl = oracle.attn_fwd(qs, ks, vs, scale=cfg.softmax_scale)
-        compare(o[b:b + 1, h * G:(h + 1) * G], lse[b:b + 1, h * G:(h + 1) * G], ro, rl,
-                f"{cfg.name} b={b} h={h}")
+        compare(o[b:b + 1], lse[b:b + 1], ro, rl, f"{cfg.name} b={b}")
 
 
 def test_decode_capturable_in_cuda_graph():

@@ -18,7 +18,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libattn_b200.so")
 SOURCES = ["attn_api.cu", "attn_kernels.cu", "attn_prefill.cu", "attn_noalloc.cu", "attn_backward.cu"]
-HEADERS = ["attn_params.h", "attn_bwd_params.h", "ptx.cuh", "host_once.h"]
+HEADERS = ["attn_params.h", "attn_bwd_params.h", "ptx.cuh", "host_once.h", "prefill_common.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
@@ -36,7 +36,7 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def source_digest(files=("attn_prefill.cu", "ptx.cuh", "attn_params.h")) -> str:
+def source_digest(files=("attn_prefill.cu", "prefill_common.cuh", "ptx.cuh", "attn_params.h")) -> str:
     """Digest of one kernel's sources and the flags (identifies a profiled
     build); by default the prefill kernel's."""
     h = hashlib.sha256()

@@ -24,6 +24,7 @@ cudaError_t launch_combine(const FwdParams&, cudaStream_t);
 template <int D>
 cudaError_t launch_prefill(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                            const FwdParams&, int, cudaStream_t);
+
 int* device_error_word();
 template <int D>
 cudaError_t launch_backward(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,

@@ -15,10 +15,11 @@
 //   warpgroup 0   warp 0: builds each unit's tile schedule (EMPTY / PARTIAL /
 //                 FULL per key tile and query tile, in shared memory, double
 //                 buffered) and issues the TMA loads (Q_A, Q_B, K/V ring);
-//                 warp 1: allocates tensor memory, lane 0 issues every MMA;
-//                 registers lowered to 72 per thread.
+//                 warp 1 (and warp 2 for d = 64, one per query tile):
+//                 allocate tensor memory and issue every MMA (elect.sync picks
+//                 the issuing lane); registers lowered to 80 per thread.
 //   warpgroup 1   softmax of tile A (one query row per thread = TMEM lane);
-//   warpgroup 2   softmax of tile B; registers raised to 216 per thread.
+//   warpgroup 2   softmax of tile B; registers raised to 208 per thread.
 // While warpgroup 1 turns S_A into P_A, the tensor core computes S_B and P_B V,
 // and the other way round.  Tensor memory: S_A [0,128), S_B [128,256), O_A at
 // 256, O_B at 256 + d.  P (bf16, 64 columns) is written over S when d = 128;
@@ -30,14 +31,22 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <type_traits>
 
 #include "attn_params.h"
 #include "host_once.h"
+#include "prefill_common.cuh"
 #include "ptx.cuh"
 
 namespace attn {
 namespace {
+
+using prefill::bit_get;
+using prefill::build_sched;
+using prefill::decode_unit;
+using prefill::key_bounds;
+using prefill::make_desc;
+using prefill::Unit;
+using prefill::unit_of;
 
 constexpr int kThreads = 384;
 constexpr int kRegsLow = 80;    // warpgroup 0 (producer, MMA)
@@ -46,16 +55,12 @@ constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
-constexpr int kBitWords = kMaxKvTiles / 32;
 
-struct Sched {
-  int t_lo, t_hi;   // union of the two query tiles' candidate key tiles
-  int n[2];         // non-empty key tiles per query tile
-  int last[2];      // last non-empty key tile per query tile (-1: none)
-  int pad[2];
-  uint32_t empty[2][kBitWords];
-  uint32_t full[2][kBitWords];
-};
+using Sched = prefill::Sched<128>;
+
+__device__ __forceinline__ bool tile_used(const Sched* s, int t) {
+  return prefill::tile_used<128>(s, t);
+}
 
 template <int D>
 struct Cfg {
@@ -98,224 +103,6 @@ enum : int {
   kTurn = 19,        // [2] softmax 1-x (128) -> softmax x: x may run its exponentials
   kKvBase = 21,      // k_full[S], k_empty[S], v_full[S], v_empty[S]
 };
-
-struct Unit {
-  int b, hq, hkv, bh;
-  int q0[2];        // first query row of tile A / B (within its sequence)
-  int rows[2];      // valid rows of tile A / B (0 if the tile is past Lq)
-  long long pos0[2];  // absolute position of row 0 of tile A / B
-  int Lk;           // keys of the sequence
-  int q_base, k_base;  // packed sequences: first token of the sequence in Q and in K/V
-  bool bad;         // packed sequences: out-of-range cu_seqlens (the unit is skipped)
-};
-
-__device__ __forceinline__ long long floor_div_ll(long long a, long long b) {
-  return a >= 0 ? a / b : -((-a + b - 1) / b);
-}
-
-__device__ __forceinline__ void key_bounds(const FwdParams& p, int Lk, long long pos,
-                                           long long& lo, long long& hi) {
-  lo = 0;
-  hi = (long long)Lk - 1;
-  if (p.mask_kind == kMaskCausal) {
-    hi = min(hi, pos);
-  } else if (p.mask_kind == kMaskDraftBlock) {
-    const long long bd = p.draft_block;
-    hi = min(hi, (floor_div_ll(pos, bd) + 1) * bd - 1);
-  }
-  if (p.window_l >= 0) lo = max(lo, pos - (long long)p.window_l);
-  if (p.window_r >= 0) hi = min(hi, pos + (long long)p.window_r);
-}
-
-// exp2 on the FMA pipe, to take part of the exponentials off the MUFU unit:
-// x = n + r with n = round(x) (the 1.5 * 2^23 trick), r in [-1/2, 1/2];
-// 2^r ~ q(r) = 1 + r*(c1 + r*(c2 + r*c3)), coefficients from
-// csrc/gen_exp2_poly.py (minimax relative error 1.0e-4 with q(0) = 1, so
-// integer arguments are exact); 2^n is added to the exponent field.  x is
-// clamped at -126, so the result is never exactly 0: only tiles without
-// masked keys use it.
-__device__ __forceinline__ float exp2_fma(float x) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  x = fmaxf(x, -126.0f);
-  const float t = x + kRound;
-  const float r = x - (t - kRound);
-  float q = fmaf(5.500893295e-02f, r, 2.422109544e-01f);
-  q = fmaf(q, r, 6.932829022e-01f);
-  q = fmaf(q, r, 1.0f);
-  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
-}
-
-// Which of the 128 exponentials of a row go to the FMA pipe.  Measured on
-// B200 (causal 4K d=64 and 32K d=128): any share made the kernel slower
-// (1/16: -1%, 1/8: -7%, 1/4: -10%), since the softmax is not limited by MUFU
-// throughput alone; kept switched off.
-constexpr bool kExpFmaShare = false;
-__host__ __device__ constexpr bool exp_on_fma(int i) { return (i & 7) == 3 && kExpFmaShare; }
-
-__device__ __forceinline__ bool bit_get(const uint32_t* bits, int i) {
-  return (bits[i >> 5] >> (i & 31)) & 1u;
-}
-
-// The u-th unit (0 = heaviest): pairs of query tiles, last pair first.  With
-// packed sequences, unit u is the pair `u / (B*Hq)` places before the last
-// pair of its sequence (units past a short sequence's first pair are empty).
-__device__ __forceinline__ void decode_unit(const FwdParams& p, int u, Unit& w) {
-  const int BH = p.B * p.Hq;
-  const int n_pairs = (p.q_tiles + 1) / 2;
-  w.bh = u % BH;
-  w.b = w.bh / p.Hq;
-  w.hq = w.bh % p.Hq;
-  w.hkv = w.hq / p.group;
-  int Lq = p.Lq, pair = n_pairs - 1 - u / BH;
-  w.Lk = p.Lk;
-  w.q_base = w.k_base = 0;
-  w.bad = false;
-  if (p.cu_seqlens_q != nullptr) {
-    const int cq0 = __ldg(p.cu_seqlens_q + w.b), cq1 = __ldg(p.cu_seqlens_q + w.b + 1);
-    const int ck0 = __ldg(p.cu_seqlens_k + w.b), ck1 = __ldg(p.cu_seqlens_k + w.b + 1);
-    Lq = cq1 - cq0;
-    const int pairs_b = ((Lq + 127) / 128 + 1) / 2;  // <= n_pairs when Lq <= p.Lq
-    w.bad = cq0 < 0 || cq1 < cq0 || cq1 > p.total_q || ck0 < 0 || ck1 < ck0 ||
-            ck1 > p.total_k || ck1 - ck0 > kMaxKvTiles * kBlockN || Lq > p.Lq;
-    pair = pairs_b - 1 - u / BH;
-    if (w.bad || pair < 0) {  // nothing to do: no rows in either tile
-      Lq = 0;
-      pair = 0;
-    }
-    w.Lk = w.bad ? 0 : ck1 - ck0;
-    w.q_base = w.bad ? 0 : cq0;
-    w.k_base = w.bad ? 0 : ck0;
-  }
-#pragma unroll
-  for (int x = 0; x < 2; ++x) {
-    const int q0 = (2 * pair + x) * 128;
-    w.q0[x] = q0;
-    w.rows[x] = max(0, min(128, Lq - q0));
-    w.pos0[x] = (long long)w.Lk - Lq + q0;
-  }
-}
-
-// Unit handled by CTA `cta` in round `r` (snake order), or -1.
-__device__ __forceinline__ int unit_of(const FwdParams& p, int cta, int r) {
-  const int G = gridDim.x;
-  const int idx = r * G + ((r & 1) ? (G - 1 - cta) : cta);
-  return idx < p.n_units ? idx : -1;
-}
-
-// Whole warp: classify the key tiles of unit w into sched.
-__device__ void build_sched(const FwdParams& p, const Unit& w, Sched* s, int lane) {
-  long long lo_first[2], hi_first[2], lo_last[2], hi_last[2];
-  int t_lo = 0x7fffffff, t_hi = -1;
-  bool any[2];
-#pragma unroll
-  for (int x = 0; x < 2; ++x) {
-    any[x] = false;
-    lo_first[x] = hi_last[x] = 0;
-    hi_first[x] = lo_last[x] = -1;
-    if (w.rows[x] > 0) {
-      key_bounds(p, w.Lk, w.pos0[x], lo_first[x], hi_first[x]);
-      key_bounds(p, w.Lk, w.pos0[x] + w.rows[x] - 1, lo_last[x], hi_last[x]);
-      if (hi_last[x] >= lo_first[x] && hi_last[x] >= 0) {
-        any[x] = true;
-        t_lo = min(t_lo, (int)(lo_first[x] / 128));
-        t_hi = max(t_hi, (int)(hi_last[x] / 128));
-      }
-    }
-  }
-  if (t_hi < 0) {
-    t_lo = 0;
-    t_hi = -1;
-  }
-  const int ntc = t_hi - t_lo + 1;
-  const int32_t* doc_b = p.doc_ids ? p.doc_ids + (long long)w.b * p.Lk : nullptr;
-  int qdmin[2] = {0, 0}, qdmax[2] = {0, 0};
-  if (doc_b) {
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      int mn = 0x7fffffff, mx = (int)0x80000000;
-      for (int r = lane; r < w.rows[x]; r += 32) {
-        const int d = __ldg(doc_b + (w.pos0[x] + r));
-        mn = min(mn, d);
-        mx = max(mx, d);
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
-      qdmin[x] = mn;
-      qdmax[x] = mx;
-    }
-  }
-  int cnt[2] = {0, 0}, last[2] = {-1, -1};
-  for (int base = 0; base < ntc; base += 32) {
-    const int i = base + lane;
-    const long long k0 = (long long)(t_lo + i) * 128;
-    bool empty[2], full[2];
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      empty[x] = (i >= ntc) || !any[x] || k0 > hi_last[x] || k0 + 127 < lo_first[x];
-      full[x] = !empty[x] && (k0 + 128 <= w.Lk) && (lo_last[x] <= k0) &&
-                (hi_first[x] >= k0 + 127);
-    }
-    if (doc_b) {
-      for (int ww = 0; ww < 32 && base + ww < ntc; ++ww) {
-        const long long kb = (long long)(t_lo + base + ww) * 128;
-        const int kend = (int)min(kb + 128, (long long)p.Lk);
-        int mn = 0x7fffffff, mx = (int)0x80000000;
-        for (long long kk = kb + lane; kk < kend; kk += 32) {
-          const int d = __ldg(doc_b + kk);
-          mn = min(mn, d);
-          mx = max(mx, d);
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        if (lane == ww) {
-#pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (mx < qdmin[x] || mn > qdmax[x]) empty[x] = true;
-            if (!(mn == mx && qdmin[x] == qdmax[x] && mn == qdmin[x])) full[x] = false;
-          }
-        }
-      }
-    }
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      const uint32_t eb = __ballot_sync(0xffffffffu, empty[x]);
-      const uint32_t fb = __ballot_sync(0xffffffffu, full[x] && !empty[x]);
-      if (lane == 0) {
-        s->empty[x][base >> 5] = eb;
-        s->full[x][base >> 5] = fb;
-      }
-      cnt[x] += __popc(~eb);
-      if (~eb) last[x] = t_lo + base + 31 - __clz(~eb);
-    }
-  }
-  if (lane == 0) {
-    s->t_lo = t_lo;
-    s->t_hi = t_hi;
-    s->n[0] = cnt[0];
-    s->n[1] = cnt[1];
-    s->last[0] = last[0];
-    s->last[1] = last[1];
-  }
-}
-
-__device__ __forceinline__ bool tile_used(const Sched* s, int t) {
-  const int i = t - s->t_lo;
-  return !(bit_get(s->empty[0], i) && bit_get(s->empty[1], i));
-}
-
-// Shared-memory descriptors (128-byte swizzle, 1024-byte stride between 8-row
-// groups): the high word is the same for every operand here, the low word
-// holds the start address and the leading offset (16-byte units).
-constexpr uint32_t kDescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
-
-__device__ __forceinline__ uint64_t make_desc(uint32_t addr, uint32_t lbo_bytes) {
-  const uint32_t lo = ((addr >> 4) & 0x3FFFu) | ((lbo_bytes >> 4) << 16);
-  return ((uint64_t)kDescHi << 32) | lo;
-}
 
 template <int D>
 __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int kk) {
@@ -919,8 +706,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The exponentials of pair i are issued kAhead pairs before their sum
         // and bf16 packing, so the MUFU results are ready when those read them
         // and one warp keeps the unit fed (measured: 4 pairs ahead is best).
-        auto emit_p = [&](auto fma_share) {
-          constexpr bool kShare = decltype(fma_share)::value;
+        ok = ptx::mbar_wait_a(bar_my_turn, (uint32_t)turns & 1u, abort_flag, err,
+                              kDevErrTimeoutSoftmax);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ++turns;
+        {
           constexpr int kAhead = 4;
           float e0[kAhead], e1[kAhead];
 #pragma unroll
@@ -940,25 +731,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int i0 = 2 * i, i1 = i0 + 1;
               float a0, a1;
               ptx::fma2_bc(a0, a1, sv[i0], sv[i1], c_s, -m_use);  // s * c - m, two at once
-              e0[i % kAhead] = (kShare && exp_on_fma(i0)) ? exp2_fma(a0) : ptx::ex2(a0);
-              e1[i % kAhead] = (kShare && exp_on_fma(i1)) ? exp2_fma(a1) : ptx::ex2(a1);
+              e0[i % kAhead] = ptx::ex2(a0);
+              e1[i % kAhead] = ptx::ex2(a1);
             }
           }
-        };
-        ok = ptx::mbar_wait_a(bar_my_turn, (uint32_t)turns & 1u, abort_flag, err,
-                              kDevErrTimeoutSoftmax);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        ++turns;
-        // One copy of the loop in the instruction stream: a second copy (for
-        // PARTIAL tiles) measured 10% slower through instruction-cache misses.
-        if constexpr (kExpFmaShare) {
-          if (full)
-            emit_p(std::true_type{});  // FULL tiles may send exponentials to the FMA pipe
-          else
-            emit_p(std::false_type{});  // PARTIAL tiles keep exact zeros at masked keys
-        } else {
-          emit_p(std::false_type{});
         }
         ptx::mbar_arrive_a(bar_other_turn);
 #pragma unroll

@@ -262,6 +262,26 @@ __device__ __forceinline__ void mma_pv_chain8(uint32_t d_tmem, uint32_t a_tmem, 
       : "memory");
 }
 
+//   O (+)= P V over 64 keys: 4 MMAs, A = P in TMEM (8 columns per step),
+//   B = V in shared memory (descriptor start address + 2048 bytes per step).
+__device__ __forceinline__ void mma_pv_chain4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p, one;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.u32 one, 0, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.u32 a, %1, 8;   add.s64 b, %2, 128;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t"
+      "add.u32 a, %1, 16;  add.s64 b, %2, 256;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t"
+      "add.u32 a, %1, 24;  add.s64 b, %2, 384;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 //   S = Q K^T with d = 64: 4 MMAs, both operands K-major in one 128-byte swizzle
 //   atom (descriptor start address + 32 bytes per step).
 __device__ __forceinline__ void mma_qk_chain_d64(uint32_t d_tmem, uint64_t a_desc,
@@ -386,6 +406,23 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
+// Named barrier `id` over 256 threads that also ORs a flag across them: every
+// participant gets true if any of them passed bad = true.  All participants
+// must reach the same sequence of meetings (there is no timeout here: the
+// callers keep their meeting counts equal on every path, aborts included).
+__device__ __forceinline__ bool pair_meet_any(int id, bool bad) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred b, a;\n\t"
+      "setp.ne.u32 b, %1, 0;\n\t"
+      "bar.red.or.pred a, %2, 256, b;\n\t"
+      "selp.u32 %0, 1, 0, a;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)bad), "r"(id)
+      : "memory");
+  return out != 0;
+}
+
 // ------------------------------------------------------------ math helpers
 // Hardware base-2 exponential and logarithm (MUFU), flush-to-zero.
 __device__ __forceinline__ float ex2(float x) {
@@ -439,6 +476,24 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Maximum of 128 values: sixteen independent chains of two-input max, then a tree.
+__device__ __forceinline__ float row_max128(const float (&v)[128]) {
+  float m[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) m[j] = fmaxf(v[j], v[16 + j]);
+#pragma unroll
+  for (int i = 32; i < 128; i += 16) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) m[j] = fmaxf(m[j], v[i + j]);
+  }
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+    for (int j = 0; j < w; ++j) m[j] = fmaxf(m[j], m[j + w]);
+  }
+  return m[0];
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` lands in the low half.

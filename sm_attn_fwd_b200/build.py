@@ -17,7 +17,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libattn_b200.so")
-SOURCES = ["attn_api.cu", "attn_kernels.cu", "attn_prefill.cu", "attn_noalloc.cu", "attn_backward.cu"]
+SOURCES = ["attn_api.cu", "attn_kernels.cu", "attn_prefill.cu", "attn_short.cu", "attn_noalloc.cu",
+           "attn_backward.cu"]
 HEADERS = ["attn_params.h", "attn_bwd_params.h", "ptx.cuh", "host_once.h", "prefill_common.cuh"]
 
 NVCC_FLAGS = [

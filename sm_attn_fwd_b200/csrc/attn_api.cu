@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -30,6 +31,9 @@ template <int D>
 cudaError_t launch_backward(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
                             const CUtensorMap&, const BwdParams&, cudaStream_t);
 cudaError_t launch_selftest_wait(cudaStream_t stream);
+template <int D>
+cudaError_t launch_short(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
+                         const FwdParams&, int, cudaStream_t);
 }  // namespace attn
 
 namespace {
@@ -194,6 +198,59 @@ size_t ws_lse_offset(const SplitPlan& pl, long long nrows, int d) {
 
 }  // namespace
 
+namespace {
+
+// Short-query plan: taken when Lq <= 128, the row tiles of all (b, kv head)
+// are fewer than twice the SM count, and the key range that any query row can
+// see under the mask (before document ids; the lower and upper bounds of a
+// row's interval never decrease with its position) spans at least 4 key tiles.
+// The cluster of a row tile splits that range into `cluster` chunks of whole
+// 128-key tiles, at most 8 CTAs per cluster and at least 8 tiles per CTA.
+struct ShortPlan {
+  int row_tiles, units, key_lo, chunk, cluster;
+};
+
+bool plan_short(int B, int Hq, int Hkv, int Lq, int Lk, int mask_kind, int wl, int wr, int bd,
+                ShortPlan* sp) {
+  if (Lq > kBlockM) return false;
+  const long long group = Hq / Hkv;
+  const long long row_tiles = ceil_div(group * Lq, kBlockM);
+  const long long units = (long long)B * Hkv * row_tiles;
+  const int sms = num_sms();
+  if (units >= 2LL * sms || units > kMaxGridY) return false;
+  // union of the rows' key intervals: positions Lk - Lq .. Lk - 1
+  const long long p_lo = (long long)Lk - Lq, p_hi = (long long)Lk - 1;
+  long long lo = 0, hi = (long long)Lk - 1;
+  if (mask_kind == ATTN_MASK_CAUSAL) {
+    hi = std::min(hi, p_hi);
+  } else if (mask_kind == ATTN_MASK_DRAFT_BLOCK) {
+    const long long blk = p_hi >= 0 ? p_hi / bd : -((-p_hi + bd - 1) / bd);
+    hi = std::min(hi, (blk + 1) * bd - 1);
+  }
+  if (wl >= 0) lo = std::max(lo, p_lo - wl);
+  if (wr >= 0) hi = std::min(hi, p_hi + wr);
+  if (hi < lo) return false;  // no row sees a key: the persistent kernel writes the empty rows
+  const long long t0 = lo / kBlockN, t1 = hi / kBlockN;
+  const long long tiles = t1 - t0 + 1;
+  // A few tiles per head are cheaper in the persistent kernel.  A cluster CTA
+  // costs several microseconds of start-up and cold loads, so the key range is
+  // split only into chunks of at least kMinTilesPerCta tiles.
+  constexpr long long kMinTiles = 4, kMinTilesPerCta = 8;
+  if (tiles < kMinTiles) return false;
+  long long cluster = std::min<long long>(8, ceil_div(2LL * sms, units));
+  cluster = std::max<long long>(1, std::min(cluster, tiles / kMinTilesPerCta));
+  const long long per = ceil_div(tiles, cluster);
+  cluster = ceil_div(tiles, per);
+  sp->row_tiles = (int)row_tiles;
+  sp->units = (int)units;
+  sp->key_lo = (int)(t0 * kBlockN);
+  sp->chunk = (int)(per * kBlockN);
+  sp->cluster = (int)cluster;
+  return true;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* attn_status_string(attn_status_t s) {
@@ -250,14 +307,30 @@ static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void
   p.err = error_word_for_current_device();
   if (!p.err) return ATTN_ERR_CUDA;
 
-  CUtensorMap tq, tk, tv;
-  const uint64_t dq[3] = {(uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq};
-  const uint64_t dk[3] = {(uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv};
-  if (!encode_bf16(&tq, q, 3, dq) || !encode_bf16(&tk, k, 3, dk) || !encode_bf16(&tv, v, 3, dk))
-    return ATTN_ERR_CUDA;
-
-  const int grid = (int)(n_units < num_sms() ? n_units : num_sms());
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  CUtensorMap tq, tk, tv;
+  const uint64_t dk[3] = {(uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv};
+  if (!encode_bf16(&tk, k, 3, dk) || !encode_bf16(&tv, v, 3, dk)) return ATTN_ERR_CUDA;
+
+  // Short queries: a query tile per (b, kv head) leaves most SMs idle in the
+  // persistent kernel, so a cluster per row tile splits the visible keys.
+  ShortPlan sp;
+  if (!alibi_slopes && plan_short(B, Hq, Hkv, Lq, Lk, mask_kind, window_l, window_r,
+                                  p.draft_block, &sp)) {
+    p.row_tiles = sp.row_tiles;
+    p.key_lo = sp.key_lo;
+    p.chunk = sp.chunk;
+    p.nsplit = sp.cluster;
+    const uint64_t dq2[2] = {(uint64_t)d, (uint64_t)B * Hq * Lq};
+    if (!encode_bf16(&tq, q, 2, dq2)) return ATTN_ERR_CUDA;
+    cudaError_t e = d == 64 ? attn::launch_short<64>(tq, tk, tv, p, sp.units, st)
+                            : attn::launch_short<128>(tq, tk, tv, p, sp.units, st);
+    return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  }
+
+  const uint64_t dq[3] = {(uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq};
+  if (!encode_bf16(&tq, q, 3, dq)) return ATTN_ERR_CUDA;
+  const int grid = (int)(n_units < num_sms() ? n_units : num_sms());
   cudaError_t e = d == 64 ? attn::launch_prefill<64>(tq, tk, tv, p, grid, st)
                           : attn::launch_prefill<128>(tq, tk, tv, p, grid, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

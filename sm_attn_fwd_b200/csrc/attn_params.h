@@ -56,6 +56,8 @@ struct FwdParams {
   int page_size;               // keys per page (power of two, >= 16)
   int pages_per_seq;           // row length of block_table; Lk = pages_per_seq * page_size
   int num_pages;               // pages in the pool
+  // short-query prefill (one cluster per row tile splits the visible keys)
+  int key_lo;                  // first key of the cluster's range (multiple of kBlockN)
 };
 
 }  // namespace attn

@@ -288,28 +288,37 @@ def run_alibi(cfg, timer, steps, warmup, stream):
     return ms, algorithmic_flops(cfg, visible_pairs(cfg))
 
 
-def run_backward(cfg, timer, steps, warmup, stream):
-    """attn_bwd on a prefill workload (d = 64).  Work: the two score GEMMs and three
-    gradient GEMMs of 2*d flop per visible pair each, 10*d*pairs in all."""
+def run_backward(cfg, timer, steps, warmup, stream, with_forward=False):
+    """attn_bwd on a prefill workload.  Work: the two score GEMMs and three
+    gradient GEMMs of 2*d flop per visible pair each, 10*d*pairs in all; with
+    the forward in the same step (a training step's attention), 14*d*pairs."""
     import sm_attn_fwd_b200 as ab
     inp = device_inputs(cfg)
     g = torch.Generator()
     g.manual_seed(cfg.seed + 1000)
     dout = torch.randn(inp.q.shape, generator=g).to(torch.bfloat16).cuda()
     torch.cuda.synchronize()
-    o, lse = ab.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask,
-                         stream=stream)
+    o = torch.empty_like(inp.q)
+    lse = torch.empty(cfg.B, cfg.Hq, cfg.Lq, dtype=torch.float32, device="cuda")
+    ab.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask, o=o, lse=lse,
+                stream=stream)
     ws = torch.empty(ab.load_library().attn_bwd_workspace_size(cfg.B, cfg.Hq, cfg.Lq, cfg.d),
                      dtype=torch.uint8, device="cuda")
     dq, dk, dv = torch.empty_like(inp.q), torch.empty_like(inp.k), torch.empty_like(inp.v)
-    fn = lambda: ab.attn_bwd(inp.q, inp.k, inp.v, o, lse, dout, scale=cfg.softmax_scale,  # noqa: E731
-                             mask=cfg.mask, workspace=ws, dq=dq, dk=dk, dv=dv, stream=stream)
+
+    def fn():
+        if with_forward:
+            ab.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask=cfg.mask, o=o, lse=lse,
+                        stream=stream)
+        ab.attn_bwd(inp.q, inp.k, inp.v, o, lse, dout, scale=cfg.softmax_scale, mask=cfg.mask,
+                    workspace=ws, dq=dq, dk=dk, dv=dv, stream=stream)
+
     ms = timer.time(fn, steps, warmup)
     st, bits = ab.attn_get_device_error(stream)
     if st != ab.ATTN_OK:
         raise RuntimeError(f"device error after attn_bwd on {cfg.name}: {st} {bits}")
     pairs = visible_pairs(cfg) * cfg.Hq
-    return ms, 10.0 * cfg.d * pairs
+    return ms, (14.0 if with_forward else 10.0) * cfg.d * pairs
 
 
 # Packed sequences: 16 documents with lengths drawn uniformly from [128, 4096]
@@ -592,12 +601,19 @@ def main():
                                                    "frac_of_bf16_peak": tf / peaks["bf16_tflops"],
                                                    "algorithmic_flop": fl6}
             if args.backward:
-                ms7, fl7 = run_backward(HEADLINE, timer, max(5, args.steps // 10), 3, stream)
-                med = statistics.median(ms7)
-                tf = fl7 / (med * 1e9)
-                workloads[HEADLINE.name + "_backward"] = {
-                    "ms_median": med, "ms_min": min(ms7), "TFLOP/s": tf,
-                    "frac_of_bf16_peak": tf / peaks["bf16_tflops"], "algorithmic_flop": fl7}
+                bwd_legs = [(HEADLINE.name + "_backward", HEADLINE, False),
+                            (HEADLINE.name + "_train_fwd_bwd", HEADLINE, True),
+                            (HEADLINE.name.replace("d64", "d128") + "_backward",
+                             HEADLINE.with_(d=128, name=HEADLINE.name.replace("d64", "d128")),
+                             False)]
+                for leg, bcfg, with_fwd in bwd_legs:
+                    ms7, fl7 = run_backward(bcfg, timer, max(5, args.steps // 10), 3, stream,
+                                            with_forward=with_fwd)
+                    med = statistics.median(ms7)
+                    tf = fl7 / (med * 1e9)
+                    workloads[leg] = {
+                        "ms_median": med, "ms_min": min(ms7), "TFLOP/s": tf,
+                        "frac_of_bf16_peak": tf / peaks["bf16_tflops"], "algorithmic_flop": fl7}
             ms5, fl5, lens5 = run_varlen(timer, max(5, args.steps // 10), 3, stream)
             med = statistics.median(ms5)
             tf = fl5 / (med * 1e9)

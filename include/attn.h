@@ -185,7 +185,7 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Lq, int d);
  *   k, v     [B, Hkv, Lk, d] bf16, read
  *   dq       [B, Hq, Lq, d] bf16, written;  dk, dv  [B, Hkv, Lk, d] bf16, written
  *   B, Hq, Hkv, Lq, Lk, scale, mask_kind, window_l, window_r, draft_block,
- *   doc_ids  as for attn_fwd; d = 64 (else UNSUPPORTED)
+ *   doc_ids  as for attn_fwd; d in {64, 128} (else UNSUPPORTED)
  *   workspace  device memory, 256-byte aligned, >= attn_bwd_workspace_size bytes,
  *            owned by the caller, not shared with a concurrent call
  *   stream   cudaStream_t; the call enqueues a memset and three kernels

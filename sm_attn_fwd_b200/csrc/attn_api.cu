@@ -438,7 +438,7 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   if (window_l < -1 || window_r < -1) return ATTN_ERR_INVALID_ARG;
   if (mask_kind == ATTN_MASK_DRAFT_BLOCK && draft_block < 1) return ATTN_ERR_INVALID_ARG;
   if (doc_ids && (!aligned(doc_ids, 4) || Lq > Lk)) return ATTN_ERR_INVALID_ARG;
-  if (d != 64) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if ((long long)B * Hkv > kMaxGridY) return ATTN_ERR_UNSUPPORTED;
   const size_t need = attn_bwd_workspace_size(B, Hq, Lq, d);
   if (need == 0 || ws_bytes < need) return ATTN_ERR_WORKSPACE;
@@ -480,7 +480,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
     return ATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(p.dq_acc, 0, rows * (size_t)d * 4, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  cudaError_t e = attn::launch_backward<64>(tq, tk, tv, tdo, p, st);
+  cudaError_t e = d == 64 ? attn::launch_backward<64>(tq, tk, tv, tdo, p, st)
+                          : attn::launch_backward<128>(tq, tk, tv, tdo, p, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

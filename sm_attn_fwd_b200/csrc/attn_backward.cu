@@ -22,8 +22,15 @@
 //              dS^T to shared memory; then, one query per thread, the dQ tile
 //              is reduced into an fp32 accumulator in global memory; at the end
 //              dK (times scale) and dV are stored as bf16.
-// Tensor memory (512 columns, d = 64): S^T / P^T [0,128), dP^T / dS^T
-// [128,256), dV [256,320), dK [320,384), dQ tile [384,448).
+// Tensor memory (512 columns).  d = 64: S^T / P^T [0,128), dP^T / dS^T
+// [128,256), dV [256,320), dK [320,384), dQ tile [384,448).  d = 128: dV
+// [256,384), dK [384,512); P^T and dS^T (bf16) take the lower 64 columns of
+// S^T and dP^T, and the dQ tile (fp32, 128 columns) is computed as two
+// 64-column halves into the freed upper halves, [64,128) and [192,256).
+// With d = 64, Q, dO and the row statistics are double-buffered: the next
+// query tile's loads, S^T and dP^T run while the softmax warps reduce this
+// tile's dQ.  (With d = 128 the second buffers do not fit in shared memory,
+// and S^T of the next tile must wait for the dQ read-out anyway.)
 // Small kernels before and after: D_i, and dQ from its fp32 accumulator.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -45,26 +52,30 @@ constexpr float kLog2eB = 1.44269504088896340736f;
 
 template <int D>
 struct BwdCfg {
+  static constexpr int kQBufs = (D == 64) ? 2 : 1;   // buffers of Q, dO and row statistics
   static constexpr int kAtomBytes = 128 * 128;       // one 64-column atom of a 128-row tile
   static constexpr int kTileBytes = 128 * D * 2;     // one Q, K, V or dO tile
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kTileBytes;
-  static constexpr int kOffQ = kOffV + kTileBytes;
-  static constexpr int kOffDO = kOffQ + kTileBytes;
-  static constexpr int kOffDS = kOffDO + kTileBytes;  // dS^T: [128 keys][128 queries] bf16
-  static constexpr int kOffStat = kOffDS + 2 * kAtomBytes;
-  static constexpr int kOffBar = kOffStat + 3 * 128 * 4;  // lse2, dsum, qdoc
-  static constexpr int kNumBars = 8;
+  static constexpr int kOffQ = kOffV + kTileBytes;          // [kQBufs]
+  static constexpr int kOffDO = kOffQ + kQBufs * kTileBytes;  // [kQBufs]
+  static constexpr int kOffDS = kOffDO + kQBufs * kTileBytes;  // dS^T: [128 keys][128 queries] bf16
+  static constexpr int kOffStat = kOffDS + 2 * kAtomBytes;     // [kQBufs] x (lse2, dsum, qdoc)
+  static constexpr int kOffBar = kOffStat + kQBufs * 3 * 128 * 4;
+  static constexpr int kNumBars = 12;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
   // at least 120 KB, so one CTA per SM holds the whole tensor memory
   static constexpr int kSmemAlloc = (kSmemBytes + 1024 > 120 * 1024) ? kSmemBytes + 1024 : 120 * 1024;
-  // tensor-memory columns
-  static constexpr uint32_t kST = 0, kDPT = 128, kDV = 256, kDK = 256 + D, kDQ = 256 + 2 * D;
+  static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
+  // tensor-memory columns (dQ: two 64-column halves for d = 128)
+  static constexpr uint32_t kST = 0, kDPT = 128, kDV = 256, kDK = 256 + D;
+  static constexpr uint32_t kDQ0 = (D == 64) ? 384u : 64u;
+  static constexpr uint32_t kDQ1 = (D == 64) ? 416u : 192u;  // columns of d = 32.. or 64..
 };
 
-enum : int { kBarKv = 0, kBarQFull, kBarQEmpty, kBarSFull, kBarPFull, kBarDqFull, kBarDqFree,
-             kBarAcc };
+enum : int { kBarKv = 0, kBarQFull, kBarQFull1, kBarQEmpty, kBarQEmpty1, kBarSFull, kBarPFull,
+             kBarDqFull, kBarDqFree, kBarAcc };
 
 __device__ __forceinline__ uint64_t bdesc(uint32_t addr, uint32_t lbo_bytes) {
   return ptx::smem_desc_sw128(addr, lbo_bytes, 1024);
@@ -138,7 +149,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p) {
   using C = BwdCfg<D>;
-  static_assert(D == 64, "tensor memory holds S^T, dP^T, dV, dK and a dQ tile for d = 64");
+  constexpr int QB = C::kQBufs;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -147,9 +158,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sq = ptx::smem_u32(smem + C::kOffQ);
   const uint32_t sdo = ptx::smem_u32(smem + C::kOffDO);
   const uint32_t sds = ptx::smem_u32(smem + C::kOffDS);
-  float* lse2_s = reinterpret_cast<float*>(smem + C::kOffStat);
-  float* dsum_s = lse2_s + 128;
-  int* qdoc_s = reinterpret_cast<int*>(dsum_s + 128);
+  // row statistics of buffer slot: lse2 [128], dsum [128], qdoc [128]
+  float* stat_s = reinterpret_cast<float*>(smem + C::kOffStat);
   const uint32_t bar0 = ptx::smem_u32(smem + C::kOffBar);
   auto BAR = [bar0](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
@@ -170,8 +180,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ptx::prefetch_tmap(&tm_do);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     ptx::mbar_init(&bars[kBarKv], 1);
-    ptx::mbar_init(&bars[kBarQFull], 1);
-    ptx::mbar_init(&bars[kBarQEmpty], 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars[kBarQFull + i], 1);
+      ptx::mbar_init(&bars[kBarQEmpty + i], 1);
+    }
     ptx::mbar_init(&bars[kBarSFull], 1);
     ptx::mbar_init(&bars[kBarPFull], 128);
     ptx::mbar_init(&bars[kBarDqFull], 1);
@@ -209,14 +221,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!pair_live(p, k0, q0)) continue;
       const int hq = iter_hq(it);
       const long long bh = (long long)b * p.Hq + hq;
-      if (n > 0) {
-        ok = ptx::mbar_wait_a(BAR(kBarQEmpty), (uint32_t)(n - 1) & 1u, abort_flag, err,
+      const int slot = n % QB;
+      if (n >= QB) {  // the slot's previous tile has been used up
+        ok = ptx::mbar_wait_a(BAR(kBarQEmpty + slot), (uint32_t)(n / QB - 1) & 1u, abort_flag, err,
                               kDevErrTimeoutProducer);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
       // row statistics of the query tile: LSE in base 2 (+inf for rows past Lq
       // or with no visible key, so their P is 0), D, and the rows' documents
+      float* lse2_s = stat_s + slot * 384;
+      float* dsum_s = lse2_s + 128;
+      int* qdoc_s = reinterpret_cast<int*>(dsum_s + 128);
       for (int r = lane; r < 128; r += 32) {
         const int qi = q0 + r;
         float l2 = INFINITY, dd = 0.0f;
@@ -233,10 +249,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx_a(BAR(kBarQFull), 2 * kTx);
+        ptx::mbar_arrive_expect_tx_a(BAR(kBarQFull + slot), 2 * kTx);
         for (int a = 0; a < D / 64; ++a) {
-          ptx::tma_load_3d_a(sq + a * C::kAtomBytes, &tm_q, BAR(kBarQFull), a * 64, q0, (int)bh);
-          ptx::tma_load_3d_a(sdo + a * C::kAtomBytes, &tm_do, BAR(kBarQFull), a * 64, q0, (int)bh);
+          ptx::tma_load_3d_a(sq + slot * C::kTileBytes + a * C::kAtomBytes, &tm_q,
+                             BAR(kBarQFull + slot), a * 64, q0, (int)bh);
+          ptx::tma_load_3d_a(sdo + slot * C::kTileBytes + a * C::kAtomBytes, &tm_do,
+                             BAR(kBarQFull + slot), a * 64, q0, (int)bh);
         }
       }
       ++n;
@@ -245,42 +263,59 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (lane == 0) {
       int dummy = 0;
       ptx::mbar_wait_a(BAR(kBarKv), 0, &dummy, nullptr, 0);
-      if (n > 0) {
+      for (int jj = max(0, n - QB); jj < n; ++jj) {
         dummy = 0;
-        ptx::mbar_wait_a(BAR(kBarQFull), (uint32_t)(n - 1) & 1u, &dummy, nullptr, 0);
+        ptx::mbar_wait_a(BAR(kBarQFull + jj % QB), (uint32_t)(jj / QB) & 1u, &dummy, nullptr, 0);
       }
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issue
     constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, 0, 0);   // K-major A and B
     constexpr uint32_t kIdAcc = ptx::idesc_bf16_f32(128, D, 0, 1);   // A from TMEM, B MN-major
-    constexpr uint32_t kIdDq = ptx::idesc_bf16_f32(128, D, 1, 1);    // A and B MN-major
+    constexpr uint32_t kIdDq = ptx::idesc_bf16_f32(128, 64, 1, 1);   // A and B MN-major, 64 of d
     bool ok = ptx::mbar_wait_a(BAR(kBarKv), 0, abort_flag, err, kDevErrTimeoutMma);
     ok = __all_sync(0xffffffffu, ok);
     int n = 0;
     for (int it = 0; it < n_iter && ok; ++it) {
       if (!pair_live(p, k0, iter_q0(it))) continue;
-      ok = ptx::mbar_wait_a(BAR(kBarQFull), (uint32_t)n & 1u, abort_flag, err, kDevErrTimeoutMma);
+      const int slot = n % QB;
+      const uint32_t sq_n = sq + slot * C::kTileBytes, sdo_n = sdo + slot * C::kTileBytes;
+      ok = ptx::mbar_wait_a(BAR(kBarQFull + slot), (uint32_t)(n / QB) & 1u, abort_flag, err,
+                            kDevErrTimeoutMma);
+      // d = 128: the previous dQ tile lives in the upper halves of S^T and dP^T
+      if (ok && D == 128 && n > 0)
+        ok = ptx::mbar_wait_a(BAR(kBarDqFree), (uint32_t)(n - 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutMma);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      // S^T = K Q^T and dP^T = V dO^T (d = 64: one swizzle atom, 4 MMAs each)
-      ptx::mma_qk_chain_d64(tmem + C::kST, bdesc(sk, 16), bdesc(sq, 16), kIdS);
-      ptx::mma_qk_chain_d64(tmem + C::kDPT, bdesc(sv, 16), bdesc(sdo, 16), kIdS);
+      // S^T = K Q^T and dP^T = V dO^T (over P^T and dS^T of the previous tile,
+      // which the previous dV and dK MMAs, issued before, have read)
+      if constexpr (D == 64) {
+        ptx::mma_qk_chain_d64(tmem + C::kST, bdesc(sk, 16), bdesc(sq_n, 16), kIdS);
+        ptx::mma_qk_chain_d64(tmem + C::kDPT, bdesc(sv, 16), bdesc(sdo_n, 16), kIdS);
+      } else {
+        ptx::mma_qk_chain_d128(tmem + C::kST, bdesc(sk, 16), bdesc(sq_n, 16), kIdS);
+        ptx::mma_qk_chain_d128(tmem + C::kDPT, bdesc(sv, 16), bdesc(sdo_n, 16), kIdS);
+      }
       ptx::mma_commit_warp(BAR(kBarSFull));
       // P^T, dS^T written (tensor memory and shared memory)
       ok = ptx::mbar_wait_a(BAR(kBarPFull), (uint32_t)n & 1u, abort_flag, err, kDevErrTimeoutMma);
-      if (ok && n > 0)  // the previous dQ tile has been read out
+      if (ok && D == 64 && n > 0)  // the previous dQ tile has been read out
         ok = ptx::mbar_wait_a(BAR(kBarDqFree), (uint32_t)(n - 1) & 1u, abort_flag, err,
                               kDevErrTimeoutMma);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
       const uint32_t acc = n > 0 ? 1u : 0u;
-      ptx::mma_pv_chain8(tmem + C::kDV, tmem + C::kST, bdesc(sdo, C::kAtomBytes), kIdAcc, acc);
-      ptx::mma_pv_chain8(tmem + C::kDK, tmem + C::kDPT, bdesc(sq, C::kAtomBytes), kIdAcc, acc);
-      mma_ss_chain8_mn(tmem + C::kDQ, bdesc(sds, C::kAtomBytes), bdesc(sk, C::kAtomBytes), kIdDq);
-      ptx::mma_commit_warp(BAR(kBarQEmpty));
+      ptx::mma_pv_chain8(tmem + C::kDV, tmem + C::kST, bdesc(sdo_n, C::kAtomBytes), kIdAcc, acc);
+      ptx::mma_pv_chain8(tmem + C::kDK, tmem + C::kDPT, bdesc(sq_n, C::kAtomBytes), kIdAcc, acc);
+      // dQ_tile = dS K, 64 columns of d per chain
+      mma_ss_chain8_mn(tmem + C::kDQ0, bdesc(sds, C::kAtomBytes), bdesc(sk, C::kAtomBytes), kIdDq);
+      if constexpr (D == 128)
+        mma_ss_chain8_mn(tmem + C::kDQ1, bdesc(sds, C::kAtomBytes),
+                         bdesc(sk + C::kAtomBytes, C::kAtomBytes), kIdDq);
+      ptx::mma_commit_warp(BAR(kBarQEmpty + slot));
       ptx::mma_commit_warp(BAR(kBarDqFull));
       ++n;
     }
@@ -302,6 +337,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int q0 = iter_q0(it);
       if (!pair_live(p, k0, q0)) continue;
       const int hq = iter_hq(it);
+      const float* lse2_s = stat_s + (n % QB) * 384;
+      const float* dsum_s = lse2_s + 128;
+      const int* qdoc_s = reinterpret_cast<const int*>(dsum_s + 128);
       ok = ptx::mbar_wait_a(BAR(kBarSFull), (uint32_t)n & 1u, abort_flag, err,
                             kDevErrTimeoutSoftmax);
       ok = __all_sync(0xffffffffu, ok);
@@ -360,8 +398,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float* dst = p.dq_acc + (((long long)b * p.Hq + hq) * p.Lq + qi) * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
+        // columns of d [32 cc, 32 cc + 32): first and second 64-column half
+        const uint32_t col = (cc < 2 ? C::kDQ0 : C::kDQ1) + (uint32_t)((cc & 1) * 32);
         uint32_t r[32];
-        ptx::tmem_ld32(t_row + C::kDQ + cc * 32, r);
+        ptx::tmem_ld32(t_row + (D == 64 ? C::kDQ0 + (uint32_t)(cc * 32) : col), r);
         ptx::tmem_wait_ld();
         if (qi < p.Lq) {
 #pragma unroll
@@ -452,5 +492,8 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
 template cudaError_t launch_backward<64>(const CUtensorMap&, const CUtensorMap&,
                                          const CUtensorMap&, const CUtensorMap&,
                                          const BwdParams&, cudaStream_t);
+template cudaError_t launch_backward<128>(const CUtensorMap&, const CUtensorMap&,
+                                          const CUtensorMap&, const CUtensorMap&,
+                                          const BwdParams&, cudaStream_t);
 
 }  // namespace attn

@@ -165,9 +165,12 @@ def test_attn_bwd_rejects_on_host_and_sizes_its_workspace():
     small = list(tail)
     small[13] = need - 1
     assert lib.attn_bwd(*ptrs, *small) == ab.ATTN_ERR_WORKSPACE
-    d128 = list(tail)
+    d96 = list(tail)
+    d96[5] = 96
+    assert lib.attn_bwd(*ptrs, *d96) == ab.ATTN_ERR_UNSUPPORTED
+    d128 = list(tail)                                  # d = 128 is built: its workspace is larger
     d128[5] = 128
-    assert lib.attn_bwd(*ptrs, *d128) == ab.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_bwd(*ptrs, *d128) == ab.ATTN_ERR_WORKSPACE
     bad_ws = list(tail)
     bad_ws[12] = ctypes.c_void_p(0x10010)                                       # not 256-aligned
     assert lib.attn_bwd(*ptrs, *bad_ws) == ab.ATTN_ERR_INVALID_ARG

@@ -27,20 +27,27 @@ def _check(got, ref, what):
 
 
 CASES = [
-    # seed, B, Hq, Hkv, Lq, Lk, mask, window, bd, doc
-    (1, 1, 2, 2, 128, 128, "none", (-1, -1), 1, False),
-    (2, 1, 2, 2, 256, 256, "causal", (-1, -1), 1, False),
-    (3, 2, 4, 2, 200, 333, "causal", (-1, -1), 1, False),
-    (4, 1, 2, 1, 300, 300, "none", (40, 17), 1, True),
-    (5, 1, 2, 2, 160, 400, "draft", (-1, 64), 16, False),
-    (6, 1, 8, 2, 129, 129, "causal", (50, 0), 1, False),
+    # seed, B, Hq, Hkv, Lq, Lk, mask, window, bd, doc, d
+    (1, 1, 2, 2, 128, 128, "none", (-1, -1), 1, False, 64),
+    (2, 1, 2, 2, 256, 256, "causal", (-1, -1), 1, False, 64),
+    (3, 2, 4, 2, 200, 333, "causal", (-1, -1), 1, False, 64),
+    (4, 1, 2, 1, 300, 300, "none", (40, 17), 1, True, 64),
+    (5, 1, 2, 2, 160, 400, "draft", (-1, 64), 16, False, 64),
+    (6, 1, 8, 2, 129, 129, "causal", (50, 0), 1, False, 64),
+    (7, 1, 2, 2, 640, 640, "causal", (-1, -1), 1, False, 64),    # many query tiles per key tile
+    (11, 1, 2, 2, 128, 128, "none", (-1, -1), 1, False, 128),
+    (12, 1, 2, 2, 256, 256, "causal", (-1, -1), 1, False, 128),
+    (13, 2, 4, 2, 200, 333, "causal", (-1, -1), 1, False, 128),
+    (14, 1, 2, 1, 300, 300, "none", (40, 17), 1, True, 128),
+    (15, 1, 2, 2, 160, 400, "draft", (-1, 64), 16, False, 128),
+    (16, 1, 8, 2, 129, 129, "causal", (50, 0), 1, False, 128),
+    (17, 1, 2, 2, 640, 640, "causal", (-1, -1), 1, False, 128),
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=lambda c: f"s{c[0]}_{c[6]}_lq{c[4]}_lk{c[5]}")
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"s{c[0]}_{c[6]}_lq{c[4]}_lk{c[5]}_d{c[10]}")
 def test_backward_matches_oracle(case):
-    seed, B, Hq, Hkv, Lq, Lk, mask, window, bd, doc = case
-    d = 64
+    seed, B, Hq, Hkv, Lq, Lk, mask, window, bd, doc, d = case
     q, k, v, doc_ids, _ = random_case(seed, B, Hq, Hkv, Lq, Lk, d, doc_split=doc, n_docs=3)
     do = torch.randn(B, Hq, Lq, d, generator=torch.Generator().manual_seed(seed + 100))
     do = do.to(torch.bfloat16)
@@ -59,8 +66,8 @@ def test_backward_matches_oracle(case):
 
 
 def test_backward_rejects_on_host():
-    q = torch.zeros(1, 2, 64, 128, dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros(1, 2, 64, 96, dtype=torch.bfloat16, device="cuda")
     lse = torch.zeros(1, 2, 64, dtype=torch.float32, device="cuda")
     with pytest.raises(ab.AttnError) as e:
-        ab.attn_bwd(q, q, q, q, lse, q)               # d = 128 not built
+        ab.attn_bwd(q, q, q, q, lse, q)               # d = 96 not built
     assert e.value.status == ab.ATTN_ERR_UNSUPPORTED

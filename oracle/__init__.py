@@ -65,6 +65,10 @@ def _load():
             lib.oracle_attn_rows_alibi.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, i32,
                                                    i32, i32, i32, P, P, P, i64, P, P, i32]
             lib.oracle_attn_rows_alibi.restype = i32
+            lib.oracle_attn_rows_relbias.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64,
+                                                     i32, i32, i32, i32, P, P, i32, P, i64, P, P,
+                                                     i32]
+            lib.oracle_attn_rows_relbias.restype = i32
             lib.oracle_decode_partials.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                                    i32, i32, P, P, i32]
             lib.oracle_decode_partials.restype = i32
@@ -140,14 +144,16 @@ def count_pairs(B, Lq, Lk, *, mask="none", window=(-1, -1), draft_block=1, doc_i
 
 
 def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
-             doc_ids=None, kv_lens=None, rows=None, nthreads=None, alibi_slopes=None):
+             doc_ids=None, kv_lens=None, rows=None, nthreads=None, alibi_slopes=None,
+             rel_bias=None):
     """Dense masked attention in double.
 
     q: [B, Hq, Lq, d] bf16; k, v: [B, Hkv, Lk, d] bf16.  Returns (O, LSE) as
     float64 numpy arrays, shaped [B, Hq, Lq, d] / [B, Hq, Lq], or [n, d] / [n]
-    when ``rows`` (flat indices (b*Hq + hq)*Lq + i) is given.  ``alibi_slopes``
-    ([Hq]) adds the ALiBi score_mod slope_h * (j - p) to every scaled score
-    (not with kv_lens).
+    when ``rows`` (flat indices (b*Hq + hq)*Lq + i) is given.  Score modifiers
+    (not with kv_lens): ``alibi_slopes`` ([Hq]) adds slope_h * (j - p) to every
+    scaled score; ``rel_bias`` = (table [Hq, 2R + 1], R) adds
+    table[h, clamp(j - p, -R, R) + R].
     """
     qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
     B, Hq, Lq, d = qb.shape
@@ -165,7 +171,20 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
         n = B * Hq * Lq
     o = np.zeros((n, d), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
-    if alibi_slopes is not None:
+    if rel_bias is not None:
+        if kl is not None or alibi_slopes is not None:
+            raise ValueError("rel_bias is not combined with kv_lens or alibi_slopes")
+        table, rmax = rel_bias
+        tb = np.ascontiguousarray(np.asarray(
+            table.cpu().numpy() if hasattr(table, "cpu") else table, dtype=np.float64))
+        if tb.shape != (Hq, 2 * int(rmax) + 1):
+            raise ValueError("rel_bias table must be [Hq, 2R + 1]")
+        rc = _load().oracle_attn_rows_relbias(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Lq, Lk, d,
+                                              float(scale), _mask_code(mask), int(window[0]),
+                                              int(window[1]), int(draft_block), _ptr(doc),
+                                              _ptr(tb), int(rmax), _ptr(rows), n, _ptr(o),
+                                              _ptr(lse), int(nthreads or max_threads()))
+    elif alibi_slopes is not None:
         if kl is not None:
             raise ValueError("alibi_slopes is not combined with kv_lens")
         sl = np.ascontiguousarray(np.asarray(
@@ -242,7 +261,7 @@ def paged_gather(pages, block_table):
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale=None, mask="none",
-                    window=(-1, -1), draft_block=1, alibi_slopes=None):
+                    window=(-1, -1), draft_block=1, alibi_slopes=None, rel_bias=None):
     """Packed sequences: the plain definition applied to each sequence on its own.
 
     q: [total_q, Hq, d] bf16, k, v: [total_k, Hkv, d] bf16 (token-major);
@@ -276,7 +295,7 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, *, scale=None, mask="no
         kb = k[k0:k1].permute(1, 0, 2).unsqueeze(0).contiguous()
         vb = v[k0:k1].permute(1, 0, 2).unsqueeze(0).contiguous()
         ob, lb = attn_fwd(qb, kb, vb, scale=scale, mask=mask, window=window,
-                          draft_block=draft_block, alibi_slopes=alibi_slopes)
+                          draft_block=draft_block, alibi_slopes=alibi_slopes, rel_bias=rel_bias)
         o[q0:q1] = ob[0].transpose(1, 0, 2)
         lse[:, q0:q1] = lb[0]
     return o, lse

@@ -154,19 +154,43 @@ int64_t oracle_count_pairs(int B, int Lq, int Lk, int mask_kind, int window_l, i
 }
 
 /*
+ * The score modifier of one query head ("FlexAttention 是什么，以及 DFlash2 之谜的
+ * 完整侦破", section 1: score_mod(score, b, h, q_idx, kv_idx) returns the new
+ * score; its examples are ALiBi, a position bias and a learnable bias).  With
+ * p the row's absolute position:
+ *   ALiBi:                 S_ij += slope * (j - p)
+ *   relative-position bias: S_ij += table[clamp(j - p, -R, R) + R]
+ * (one table row of 2R + 1 values per query head; the values may be learned).
+ */
+typedef struct {
+  double alibi_slope;     /* 0 leaves the scores as they are */
+  const double* rel_row;  /* the head's table row, or NULL */
+  int rel_max;            /* R */
+} score_mod;
+
+static double score_bias(const score_mod* sm, int j, double p_abs) {
+  double bias = sm->alibi_slope * ((double)j - p_abs);
+  if (sm->rel_row) {
+    long long delta = (long long)j - (long long)p_abs;
+    if (delta < -sm->rel_max) delta = -sm->rel_max;
+    if (delta > sm->rel_max) delta = sm->rel_max;
+    bias += sm->rel_row[delta + sm->rel_max];
+  }
+  return bias;
+}
+
+/*
  * One query row over the keys [j_lo, j_hi) that the mask allows:
  * scores, max pass, sum pass, weighted sum of V.  Writes d values to o_row
  * and returns the row's LSE (-inf when no key is allowed; o_row is then 0).
  */
 static double attend_row(const uint16_t* q_row, const uint16_t* k_head, const uint16_t* v_head,
                          int d, double scale, const mask_spec* m, int b, int i, int j_lo,
-                         int j_hi, double alibi_slope, double* s_buf, uint8_t* ok_buf,
+                         int j_hi, const score_mod* sm, double* s_buf, uint8_t* ok_buf,
                          double* q_buf, double* o_row) {
   for (int c = 0; c < d; ++c) q_buf[c] = bf16_bits_to_double(q_row[c]);
   /* scores of the row: S_ij = scale * sum_c Q_ic K_jc, then the score_mod
-     ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", section 1: score_mod(score,
-     b, h, q_idx, kv_idx), e.g. ALiBi): S_ij += slope_h * (j - p), p the row's
-     absolute position; slope 0 leaves the scores as they are */
+     (score_bias above), p the row's absolute position */
   const double p_abs = (double)(key_count(m, b) - m->Lq + i);
   int any = 0;
   for (int j = j_lo; j < j_hi; ++j) {
@@ -175,7 +199,7 @@ static double attend_row(const uint16_t* q_row, const uint16_t* k_head, const ui
     const uint16_t* k_row = k_head + (int64_t)j * d;
     double acc = 0.0;
     for (int c = 0; c < d; ++c) acc += q_buf[c] * bf16_bits_to_double(k_row[c]);
-    s_buf[j - j_lo] = scale * acc + alibi_slope * ((double)j - p_abs);
+    s_buf[j - j_lo] = scale * acc + score_bias(sm, j, p_abs);
     any = 1;
   }
   for (int c = 0; c < d; ++c) o_row[c] = 0.0;
@@ -212,8 +236,9 @@ static int check_shapes(int B, int Hq, int Hkv, int Lq, int Lk, int d) {
 static int attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
                      int Hkv, int Lq, int Lk, int d, double scale, int mask_kind, int window_l,
                      int window_r, int draft_block, const int32_t* doc_ids,
-                     const int32_t* kv_lens, const double* alibi_slopes, const int64_t* rows,
-                     int64_t nrows, double* o, double* lse, int nthreads) {
+                     const int32_t* kv_lens, const double* alibi_slopes, const double* rel_table,
+                     int rel_max, const int64_t* rows, int64_t nrows, double* o, double* lse,
+                     int nthreads) {
   if (check_shapes(B, Hq, Hkv, Lq, Lk, d)) return -1;
   mask_spec m = {B, Lq, Lk, mask_kind, window_l, window_r, draft_block, doc_ids, kv_lens};
   if (check_mask_spec(&m)) return -1;
@@ -244,8 +269,9 @@ static int attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
       const uint16_t* q_row = q + flat * d;
       const uint16_t* k_head = k + ((int64_t)b * Hkv + hkv) * Lk * d;
       const uint16_t* v_head = v + ((int64_t)b * Hkv + hkv) * Lk * d;
-      const double slope = alibi_slopes ? alibi_slopes[hq] : 0.0;
-      lse[r] = attend_row(q_row, k_head, v_head, d, scale, &m, b, i, 0, Lk, slope, s_buf, ok_buf,
+      score_mod sm = {alibi_slopes ? alibi_slopes[hq] : 0.0,
+                      rel_table ? rel_table + (int64_t)hq * (2 * rel_max + 1) : NULL, rel_max};
+      lse[r] = attend_row(q_row, k_head, v_head, d, scale, &m, b, i, 0, Lk, &sm, s_buf, ok_buf,
                           q_buf, o + r * d);
     }
     free(s_buf);
@@ -261,7 +287,7 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, in
                      const int32_t* kv_lens, const int64_t* rows, int64_t nrows, double* o,
                      double* lse, int nthreads) {
   return attn_rows(q, k, v, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
-                   draft_block, doc_ids, kv_lens, NULL, rows, nrows, o, lse, nthreads);
+                   draft_block, doc_ids, kv_lens, NULL, NULL, 0, rows, nrows, o, lse, nthreads);
 }
 
 /* The same with the ALiBi score_mod: alibi_slopes[hq] per query head. */
@@ -272,7 +298,21 @@ int oracle_attn_rows_alibi(const uint16_t* q, const uint16_t* k, const uint16_t*
                            double* o, double* lse, int nthreads) {
   if (!alibi_slopes) return -1;
   return attn_rows(q, k, v, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
-                   draft_block, doc_ids, NULL, alibi_slopes, rows, nrows, o, lse, nthreads);
+                   draft_block, doc_ids, NULL, alibi_slopes, NULL, 0, rows, nrows, o, lse,
+                   nthreads);
+}
+
+/* The same with the relative-position bias: table [Hq][2 rel_max + 1]. */
+int oracle_attn_rows_relbias(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                             int Hq, int Hkv, int Lq, int Lk, int d, double scale, int mask_kind,
+                             int window_l, int window_r, int draft_block,
+                             const int32_t* doc_ids, const double* table, int rel_max,
+                             const int64_t* rows, int64_t nrows, double* o, double* lse,
+                             int nthreads) {
+  if (!table || rel_max < 0) return -1;
+  return attn_rows(q, k, v, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
+                   draft_block, doc_ids, NULL, NULL, table, rel_max, rows, nrows, o, lse,
+                   nthreads);
 }
 
 /*
@@ -287,6 +327,7 @@ int oracle_decode_partials(const uint16_t* q, const uint16_t* k, const uint16_t*
                            const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq, int Lk,
                            int d, double scale, int chunk, int nsplit, double* o_part,
                            double* lse_part, int nthreads) {
+  const score_mod no_mod = {0.0, NULL, 0};
   if (check_shapes(B, Hq, Hkv, Lq, Lk, d) || chunk < 1 || nsplit < 1) return -1;
   if (!kv_lens) return -1;
   mask_spec m = {B, Lq, Lk, ORACLE_MASK_NONE, -1, -1, 1, NULL, kv_lens};
@@ -325,7 +366,7 @@ int oracle_decode_partials(const uint16_t* q, const uint16_t* k, const uint16_t*
         lse_part[(int64_t)s * nrows + r] =
             attend_row(q + r * d, k + ((int64_t)b * Hkv + hkv) * Lk * d,
                        v + ((int64_t)b * Hkv + hkv) * Lk * d, d, scale, &m, b, i, j_lo, j_hi,
-                       0.0, s_buf, ok_buf, q_buf, o_row);
+                       &no_mod, s_buf, ok_buf, q_buf, o_row);
       }
     }
     free(s_buf);

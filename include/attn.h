@@ -100,31 +100,41 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        void* stream);
 
 typedef enum {
-  ATTN_SCORE_MOD_NONE = 0,  /* S_ij unchanged */
-  ATTN_SCORE_MOD_ALIBI = 1  /* S_ij += slope[hq] * (j - p); params = slope[Hq] */
+  ATTN_SCORE_MOD_NONE = 0,    /* S_ij unchanged */
+  ATTN_SCORE_MOD_ALIBI = 1,   /* S_ij += slope[hq] * (j - p); params = slope[Hq] */
+  ATTN_SCORE_MOD_REL_BIAS = 2 /* S_ij += table[hq][clamp(j - p, -R, R) + R]; params = table,
+                                 arg = R */
 } attn_score_mod_kind_t;
 
 /*
  * attn_fwd_score_mod — attn_fwd with a score modifier.
  *
  * Defines ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破", section 1:
- * score_mod(score, b, h, q_idx, kv_idx) -> score, e.g. ALiBi or a position
- * bias): the scaled score S_ij of attn_fwd is replaced by the modified score
- * before the mask and the softmax; LSE is taken over the modified scores.
- *   ATTN_SCORE_MOD_ALIBI: S_ij = scale * <Q_i, K_j> + slope[hq] * (j - p), with
- *   p = Lk - Lq + i the row's absolute position and slope a caller-given
- *   per-query-head value (for example 2^(-8 (hq+1) / Hq)).
+ * score_mod(score, b, h, q_idx, kv_idx) -> score, with ALiBi, a position bias
+ * and a learnable bias as examples): the scaled score S_ij of attn_fwd is
+ * replaced by the modified score before the mask and the softmax; LSE is
+ * taken over the modified scores.  p = Lk - Lq + i is the row's absolute
+ * position.
+ *   ATTN_SCORE_MOD_ALIBI: S_ij = scale * <Q_i, K_j> + slope[hq] * (j - p),
+ *   with a caller-given per-query-head slope (for example 2^(-8 (hq+1) / Hq)).
+ *   ATTN_SCORE_MOD_REL_BIAS: S_ij = scale * <Q_i, K_j> + table[hq][clamp(j - p,
+ *   -R, R) + R]: a relative-position bias, one row of 2R + 1 values per query
+ *   head (a learned table, a fixed position bias, or a per-head constant
+ *   with R = 0); distances beyond R share the value at the end of the row.
  *
  * Arguments: those of attn_fwd, plus
  *   score_mod         one of attn_score_mod_kind_t
- *   score_mod_params  ALIBI: [Hq] fp32 device array (4-byte aligned); NONE: ignored
- * Errors: as attn_fwd; INVALID_ARG for an unknown score_mod or missing params.
+ *   score_mod_params  ALIBI: [Hq] fp32 device array; REL_BIAS: [Hq][2R + 1] fp32
+ *                     device array; both 4-byte aligned; NONE: ignored
+ *   score_mod_arg     REL_BIAS: R, 0 <= R <= 2^20; otherwise ignored
+ * Errors: as attn_fwd; INVALID_ARG for an unknown score_mod, missing params or
+ * a bad R.
  */
 attn_status_t attn_fwd_score_mod(const void* q, const void* k, const void* v, void* o,
                                  float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d,
                                  float scale, int mask_kind, int window_l, int window_r,
                                  int draft_block, const int32_t* doc_ids, int score_mod,
-                                 const float* score_mod_params, void* stream);
+                                 const float* score_mod_params, int score_mod_arg, void* stream);
 
 /*
  * attn_fwd_varlen — prefill attention forward over packed sequences.
@@ -160,6 +170,21 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
                               int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
                               float scale, int mask_kind, int window_l, int window_r,
                               int draft_block, void* stream);
+
+/*
+ * attn_fwd_varlen_score_mod — attn_fwd_varlen with a score modifier, as in
+ * attn_fwd_score_mod: p is the row's absolute position inside its own
+ * sequence (Lk_b - Lq_b + i).  Arguments: those of attn_fwd_varlen, plus
+ * score_mod, score_mod_params and score_mod_arg as for attn_fwd_score_mod.
+ */
+attn_status_t attn_fwd_varlen_score_mod(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int B, int Hq, int Hkv,
+                                        int total_q, int total_k, int max_seqlen_q, int d,
+                                        float scale, int mask_kind, int window_l, int window_r,
+                                        int draft_block, int score_mod,
+                                        const float* score_mod_params, int score_mod_arg,
+                                        void* stream);
 
 /*
  * attn_bwd_workspace_size — bytes of caller workspace attn_bwd needs:

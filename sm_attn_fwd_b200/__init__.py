@@ -26,7 +26,7 @@ __all__ = [
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
     "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_bwd", "attn_decode_splitkv",
-    "attn_decode_num_splits", "SCORE_MOD_NONE", "SCORE_MOD_ALIBI",
+    "attn_decode_num_splits", "SCORE_MOD_NONE", "SCORE_MOD_ALIBI", "SCORE_MOD_REL_BIAS",
     "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
     "EXPORTED_SYMBOLS",
@@ -44,10 +44,12 @@ MASK_CAUSAL = 1
 MASK_DRAFT_BLOCK = 2
 SCORE_MOD_NONE = 0
 SCORE_MOD_ALIBI = 1
+SCORE_MOD_REL_BIAS = 2
 _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 
 EXPORTED_SYMBOLS = (
-    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_bwd_workspace_size", "attn_bwd",
+    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_fwd_varlen_score_mod",
+    "attn_bwd_workspace_size", "attn_bwd",
     "attn_decode_num_splits", "attn_decode_workspace_size",
     "attn_decode_splitkv", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
@@ -84,7 +86,7 @@ def load_library():
                                  i32, P, P]
         lib.attn_fwd.restype = i32
         lib.attn_fwd_score_mod.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
-                                           i32, i32, i32, P, i32, P, P]
+                                           i32, i32, i32, P, i32, P, i32, P]
         lib.attn_fwd_score_mod.restype = i32
         lib.attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.attn_bwd_workspace_size.restype = sz
@@ -94,6 +96,10 @@ def load_library():
         lib.attn_fwd_varlen.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32,
                                         i32, i32, i32, i32, P]
         lib.attn_fwd_varlen.restype = i32
+        lib.attn_fwd_varlen_score_mod.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                                  i32, i32, f32, i32, i32, i32, i32, i32, P, i32,
+                                                  P]
+        lib.attn_fwd_varlen_score_mod.restype = i32
         lib.attn_decode_num_splits.argtypes = [i32] * 7 + [ctypes.POINTER(ctypes.c_int)]
         lib.attn_decode_num_splits.restype = i32
         lib.attn_decode_workspace_size.argtypes = [i32] * 7
@@ -169,17 +175,36 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
     return o, lse
 
 
-def attn_fwd_score_mod(q, k, v, *, alibi_slopes, scale=None, mask="none", window=(-1, -1),
-                       draft_block=1, doc_ids=None, o=None, lse=None, stream=None):
-    """attn_fwd with the ALiBi score_mod (see ``attn_fwd_score_mod`` in include/attn.h):
-    S_ij += alibi_slopes[hq] * (j - p).  alibi_slopes: fp32 CUDA tensor [Hq]."""
+def _score_mod_args(Hq, alibi_slopes, rel_bias):
+    """(kind, params tensor, arg) of the score modifier; at most one is given."""
+    if alibi_slopes is not None and rel_bias is not None:
+        raise ValueError("give alibi_slopes or rel_bias, not both")
+    if alibi_slopes is not None:
+        if (alibi_slopes.dtype != torch.float32 or not alibi_slopes.is_cuda
+                or not alibi_slopes.is_contiguous() or alibi_slopes.numel() != Hq):
+            raise ValueError("alibi_slopes must be a contiguous fp32 CUDA tensor [Hq]")
+        return SCORE_MOD_ALIBI, alibi_slopes, 0
+    if rel_bias is not None:
+        table, rmax = rel_bias
+        if (table.dtype != torch.float32 or not table.is_cuda or not table.is_contiguous()
+                or tuple(table.shape) != (Hq, 2 * int(rmax) + 1)):
+            raise ValueError("rel_bias table must be a contiguous fp32 CUDA tensor [Hq, 2R + 1]")
+        return SCORE_MOD_REL_BIAS, table, int(rmax)
+    return SCORE_MOD_NONE, None, 0
+
+
+def attn_fwd_score_mod(q, k, v, *, alibi_slopes=None, rel_bias=None, scale=None, mask="none",
+                       window=(-1, -1), draft_block=1, doc_ids=None, o=None, lse=None,
+                       stream=None):
+    """attn_fwd with a score modifier (see ``attn_fwd_score_mod`` in include/attn.h):
+    ALiBi, S_ij += alibi_slopes[hq] * (j - p) (fp32 CUDA tensor [Hq]), or the
+    relative-position bias rel_bias = (table, R), S_ij += table[hq, clamp(j - p, -R, R) + R]
+    (fp32 CUDA tensor [Hq, 2R + 1])."""
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_bf16(name, t)
     B, Hq, Lq, d = q.shape
     _, Hkv, Lk, _ = k.shape
-    if (alibi_slopes.dtype != torch.float32 or not alibi_slopes.is_cuda
-            or not alibi_slopes.is_contiguous() or alibi_slopes.numel() != Hq):
-        raise ValueError("alibi_slopes must be a contiguous fp32 CUDA tensor [Hq]")
+    kind, params, arg = _score_mod_args(Hq, alibi_slopes, rel_bias)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if o is None:
@@ -193,7 +218,7 @@ def attn_fwd_score_mod(q, k, v, *, alibi_slopes, scale=None, mask="none", window
     st = load_library().attn_fwd_score_mod(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
                                            Hkv, Lq, Lk, d, float(scale), mk, int(window[0]),
                                            int(window[1]), int(draft_block), _ptr(doc_ids),
-                                           SCORE_MOD_ALIBI, _ptr(alibi_slopes),
+                                           kind, _ptr(params), arg,
                                            _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_score_mod")
@@ -237,12 +262,14 @@ def attn_bwd(q, k, v, o, lse, dout, *, scale=None, mask="none", window=(-1, -1),
 
 
 def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, *, scale=None,
-                    mask="none", window=(-1, -1), draft_block=1, o=None, lse=None, stream=None):
-    """Prefill forward over packed sequences (see ``attn_fwd_varlen`` in include/attn.h).
+                    mask="none", window=(-1, -1), draft_block=1, alibi_slopes=None,
+                    rel_bias=None, o=None, lse=None, stream=None):
+    """Prefill forward over packed sequences (see ``attn_fwd_varlen`` and
+    ``attn_fwd_varlen_score_mod`` in include/attn.h).
 
     q: [total_q, Hq, d], k/v: [total_k, Hkv, d] bf16 CUDA tensors (token-major);
-    cu_seqlens_q/k: int32 CUDA tensors [B + 1].  Returns (o bf16 [total_q, Hq, d],
-    lse fp32 [Hq, total_q]).
+    cu_seqlens_q/k: int32 CUDA tensors [B + 1].  Optional score modifier as in
+    ``attn_fwd_score_mod``.  Returns (o bf16 [total_q, Hq, d], lse fp32 [Hq, total_q]).
     """
     for name, t in (("q", q), ("k", k), ("v", v)):
         _check_bf16(name, t, "[total, H, D]")
@@ -261,11 +288,12 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, *, scale=
     if lse is None:
         lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
     mk = mask if isinstance(mask, int) else _MASKS[mask]
-    st = load_library().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
-                                        _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B, Hq, Hkv, total_q,
-                                        total_k, int(max_seqlen_q), d, float(scale), mk,
-                                        int(window[0]), int(window[1]), int(draft_block),
-                                        _stream_handle(stream, q.device))
+    kind, params, arg = _score_mod_args(Hq, alibi_slopes, rel_bias)
+    st = load_library().attn_fwd_varlen_score_mod(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), B,
+        Hq, Hkv, total_q, total_k, int(max_seqlen_q), d, float(scale), mk, int(window[0]),
+        int(window[1]), int(draft_block), kind, _ptr(params), arg,
+        _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_varlen")
     return o, lse

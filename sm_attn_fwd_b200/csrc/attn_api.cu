@@ -265,10 +265,35 @@ const char* attn_status_string(attn_status_t s) {
   return "ATTN_ERR_UNKNOWN";
 }
 
+// Score modifier of a call (ALiBi slopes or a relative-position table; at most one).
+struct ScoreMod {
+  const float* alibi_slopes = nullptr;
+  const float* rel_table = nullptr;
+  int rel_max = 0;
+};
+
+// Checks the score_mod arguments of attn_fwd_score_mod / attn_fwd_varlen_score_mod.
+static attn_status_t parse_score_mod(int kind, const float* params, int arg, ScoreMod* sm) {
+  *sm = ScoreMod{};
+  if (kind == ATTN_SCORE_MOD_NONE) return ATTN_OK;
+  if (!params || !aligned(params, 4)) return ATTN_ERR_INVALID_ARG;
+  if (kind == ATTN_SCORE_MOD_ALIBI) {
+    sm->alibi_slopes = params;
+    return ATTN_OK;
+  }
+  if (kind == ATTN_SCORE_MOD_REL_BIAS) {
+    if (arg < 0 || arg > (1 << 20)) return ATTN_ERR_INVALID_ARG;
+    sm->rel_table = params;
+    sm->rel_max = arg;
+    return ATTN_OK;
+  }
+  return ATTN_ERR_INVALID_ARG;
+}
+
 static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse,
                                int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
                                int mask_kind, int window_l, int window_r, int draft_block,
-                               const int32_t* doc_ids, const float* alibi_slopes, void* stream) {
+                               const int32_t* doc_ids, const ScoreMod& sm, void* stream) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4))
@@ -288,7 +313,9 @@ static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void
   p.o = o;
   p.lse = lse;
   p.doc_ids = doc_ids;
-  p.alibi_slopes = alibi_slopes;
+  p.alibi_slopes = sm.alibi_slopes;
+  p.rel_table = sm.rel_table;
+  p.rel_max = sm.rel_max;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -315,8 +342,8 @@ static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void
   // Short queries: a query tile per (b, kv head) leaves most SMs idle in the
   // persistent kernel, so a cluster per row tile splits the visible keys.
   ShortPlan sp;
-  if (!alibi_slopes && plan_short(B, Hq, Hkv, Lq, Lk, mask_kind, window_l, window_r,
-                                  p.draft_block, &sp)) {
+  if (!sm.alibi_slopes && !sm.rel_table &&
+      plan_short(B, Hq, Hkv, Lq, Lk, mask_kind, window_l, window_r, p.draft_block, &sp)) {
     p.row_tiles = sp.row_tiles;
     p.key_lo = sp.key_lo;
     p.chunk = sp.chunk;
@@ -341,28 +368,26 @@ attn_status_t attn_fwd(const void* q, const void* k, const void* v, void* o, flo
                        int window_l, int window_r, int draft_block, const int32_t* doc_ids,
                        void* stream) {
   return fwd_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
-                   draft_block, doc_ids, nullptr, stream);
+                   draft_block, doc_ids, ScoreMod{}, stream);
 }
 
 attn_status_t attn_fwd_score_mod(const void* q, const void* k, const void* v, void* o,
                                  float* lse, int B, int Hq, int Hkv, int Lq, int Lk, int d,
                                  float scale, int mask_kind, int window_l, int window_r,
                                  int draft_block, const int32_t* doc_ids, int score_mod,
-                                 const float* score_mod_params, void* stream) {
-  if (score_mod == ATTN_SCORE_MOD_NONE)
-    return fwd_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
-                     draft_block, doc_ids, nullptr, stream);
-  if (score_mod != ATTN_SCORE_MOD_ALIBI) return ATTN_ERR_INVALID_ARG;
-  if (!score_mod_params || !aligned(score_mod_params, 4)) return ATTN_ERR_INVALID_ARG;
+                                 const float* score_mod_params, int score_mod_arg, void* stream) {
+  ScoreMod sm;
+  const attn_status_t st = parse_score_mod(score_mod, score_mod_params, score_mod_arg, &sm);
+  if (st != ATTN_OK) return st;
   return fwd_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
-                   draft_block, doc_ids, score_mod_params, stream);
+                   draft_block, doc_ids, sm, stream);
 }
 
-attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
-                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
-                              int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
-                              float scale, int mask_kind, int window_l, int window_r,
-                              int draft_block, void* stream) {
+static attn_status_t fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                                const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                                int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
+                                float scale, int mask_kind, int window_l, int window_r,
+                                int draft_block, const ScoreMod& sm, void* stream) {
   if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4) || !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
@@ -382,6 +407,9 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
   p.lse = lse;
   p.cu_seqlens_q = cu_seqlens_q;
   p.cu_seqlens_k = cu_seqlens_k;
+  p.alibi_slopes = sm.alibi_slopes;
+  p.rel_table = sm.rel_table;
+  p.rel_max = sm.rel_max;
   p.total_q = total_q;
   p.total_k = total_k;
   p.B = B;
@@ -412,6 +440,32 @@ attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void*
   cudaError_t e = d == 64 ? attn::launch_prefill<64>(tq, tk, tv, p, grid, st)
                           : attn::launch_prefill<128>(tq, tk, tv, p, grid, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status_t attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                              const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                              int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
+                              float scale, int mask_kind, int window_l, int window_r,
+                              int draft_block, void* stream) {
+  return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, total_q, total_k,
+                    max_seqlen_q, d, scale, mask_kind, window_l, window_r, draft_block,
+                    ScoreMod{}, stream);
+}
+
+attn_status_t attn_fwd_varlen_score_mod(const void* q, const void* k, const void* v, void* o,
+                                        float* lse, const int32_t* cu_seqlens_q,
+                                        const int32_t* cu_seqlens_k, int B, int Hq, int Hkv,
+                                        int total_q, int total_k, int max_seqlen_q, int d,
+                                        float scale, int mask_kind, int window_l, int window_r,
+                                        int draft_block, int score_mod,
+                                        const float* score_mod_params, int score_mod_arg,
+                                        void* stream) {
+  ScoreMod sm;
+  const attn_status_t st = parse_score_mod(score_mod, score_mod_params, score_mod_arg, &sm);
+  if (st != ATTN_OK) return st;
+  return fwd_varlen(q, k, v, o, lse, cu_seqlens_q, cu_seqlens_k, B, Hq, Hkv, total_q, total_k,
+                    max_seqlen_q, d, scale, mask_kind, window_l, window_r, draft_block, sm,
+                    stream);
 }
 
 size_t attn_bwd_workspace_size(int B, int Hq, int Lq, int d) {

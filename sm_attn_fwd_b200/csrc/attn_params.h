@@ -45,8 +45,11 @@ struct FwdParams {
   int q_tiles;       // prefill: ceil(Lq / 128)
   int n_units;       // prefill: work units (pairs of query tiles x B*Hq)
   int* err;          // device error word
-  // score_mod (prefill): ALiBi slopes [Hq] fp32, or null
+  // score_mod (prefill): ALiBi slopes [Hq] fp32, or null; or a relative-position
+  // table [Hq][2 rel_max + 1] fp32, or null
   const float* alibi_slopes;
+  const float* rel_table;
+  int rel_max;
   // packed sequences (prefill): null for the [B, H, L, d] layout
   const int32_t* cu_seqlens_q;  // [B + 1]
   const int32_t* cu_seqlens_k;  // [B + 1]

@@ -55,6 +55,7 @@ constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
+enum : int { kModNone = 0, kModAlibi = 1, kModRelBias = 2 };
 
 using Sched = prefill::Sched<128>;
 
@@ -116,9 +117,10 @@ __device__ __forceinline__ uint64_t desc_v(uint32_t tile_saddr, int kk) {
 
 }  // namespace
 
-// kAlibi: the ALiBi score_mod, S_ij += slope_h * (j - p) (p the row's absolute
-// position), with p.alibi_slopes[hq] per query head.
-template <int D, bool kAlibi>
+// kMod: the score modifier (p the row's absolute position):
+//   kModNone;  kModAlibi: S_ij += slope_h * (j - p), p.alibi_slopes[hq];
+//   kModRelBias: S_ij += table[hq][clamp(j - p, -R, R) + R], p.rel_table, R = p.rel_max.
+template <int D, int kMod>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
@@ -507,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t bar_o_done = BAR(kODone + x);
     const uint32_t bar_o_free = BAR(kOFree + x);
     const float c = p.scale_log2;
-    const float c_s = kAlibi ? 1.0f : c;  // scale still to apply to the loaded scores
+    const float c_s = kMod != kModNone ? 1.0f : c;  // scale still to apply to the loaded scores
     int ns = 0;  // S tiles consumed (global count)
     // The two softmax warpgroups take turns on the exponentials of each key
     // tile (A, B, A, B, ...), so that one loads S, finds the row max and stores
@@ -531,7 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_ok = r_row < w.rows[x];
       // ALiBi: the row's absolute position and the head's slope times log2(e)
       const long long row_pos = w.pos0[x] + r_row;
-      const float alibi2 = kAlibi ? __ldg(p.alibi_slopes + w.hq) * kLog2e : 0.0f;
+      const float alibi2 = kMod == kModAlibi ? __ldg(p.alibi_slopes + w.hq) * kLog2e : 0.0f;
+      // relative-position table of the head, centred on j - p = 0
+      const float* rel_row =
+          kMod == kModRelBias ? p.rel_table + (long long)w.hq * (2 * p.rel_max + 1) + p.rel_max
+                              : nullptr;
       int row_lo = 0, row_hi = -1;  // visible key range, clamped to [0, Lk-1]
       int row_doc = 0;
       // document ids of this batch row (warp-uniform: every lane takes part in
@@ -652,7 +658,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[i] = ((word >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
           }
         }
-        if constexpr (kAlibi) {
+        if constexpr (kMod == kModRelBias) {
+          // scores to the base-2 domain with the table's bias:
+          // s*c + table[clamp(j - p, -R, R)]*log2(e); masked scores stay -inf.
+          // A tile whose keys all lie R or more from the row on one side takes
+          // one clamped value; only tiles within R of the row look keys up.
+          const int R = p.rel_max;
+          const int dj0 = k0 - (int)row_pos;  // j - p at the tile's first key
+          if (dj0 + 127 <= -R || dj0 >= R) {
+            const float bias = __ldg(rel_row + (dj0 >= R ? R : -R)) * kLog2e;
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              ptx::fma2_bc(sv[2 * i], sv[2 * i + 1], sv[2 * i], sv[2 * i + 1], c, bias);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 128; ++i) {
+              const int delta = min(max(dj0 + i, -R), R);
+              sv[i] = fmaf(__ldg(rel_row + delta), kLog2e, sv[i] * c);
+            }
+          }
+        }
+        if constexpr (kMod == kModAlibi) {
           // scores to the base-2 domain with the bias: s*c + slope*log2(e)*(j - p);
           // masked scores stay -inf.  The max and the exponentials below then
           // use a scale of 1.
@@ -833,11 +859,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool kAlibi>
+template <int D, int kMod>
 cudaError_t launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tk,
                                   const CUtensorMap& tv, const FwdParams& p, int grid,
                                   cudaStream_t stream) {
-  auto kern = attn_prefill_kernel<D, kAlibi>;
+  auto kern = attn_prefill_kernel<D, kMod>;
   constexpr int smem = Cfg<D>::kSmemAlloc;
   static PerContextOnce once;
   const cudaError_t e = once_per_context(once, [&](int) {
@@ -851,8 +877,9 @@ cudaError_t launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tk,
 template <int D>
 cudaError_t launch_prefill(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            const FwdParams& p, int grid, cudaStream_t stream) {
-  return p.alibi_slopes ? launch_prefill_kernel<D, true>(tq, tk, tv, p, grid, stream)
-                        : launch_prefill_kernel<D, false>(tq, tk, tv, p, grid, stream);
+  if (p.alibi_slopes) return launch_prefill_kernel<D, kModAlibi>(tq, tk, tv, p, grid, stream);
+  if (p.rel_table) return launch_prefill_kernel<D, kModRelBias>(tq, tk, tv, p, grid, stream);
+  return launch_prefill_kernel<D, kModNone>(tq, tk, tv, p, grid, stream);
 }
 
 template cudaError_t launch_prefill<64>(const CUtensorMap&, const CUtensorMap&,

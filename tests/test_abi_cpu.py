@@ -141,11 +141,16 @@ def test_attn_fwd_varlen_rejects_on_host():
 def test_attn_fwd_score_mod_rejects_on_host():
     lib = ab.load_library()
     #      q  k  v  o  lse B  Hq Hkv Lq   Lk   d   scale mask wl  wr bd doc  kind params stream
-    args = [A, A, A, A, A, 2, 8, 2, 100, 100, 64, 0.125, 1, -1, -1, 1, None, 1, A, None]
-    assert lib.attn_fwd_score_mod(*args[:17], 7, A, None) == ab.ATTN_ERR_INVALID_ARG
-    assert lib.attn_fwd_score_mod(*args[:17], 1, None, None) == ab.ATTN_ERR_INVALID_ARG
-    assert lib.attn_fwd_score_mod(*args[:17], 1, ctypes.c_void_p(0x10002), None) == \
+    args = [A, A, A, A, A, 2, 8, 2, 100, 100, 64, 0.125, 1, -1, -1, 1, None, 1, A, 0, None]
+    assert lib.attn_fwd_score_mod(*args[:17], 7, A, 0, None) == ab.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_score_mod(*args[:17], 1, None, 0, None) == ab.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_score_mod(*args[:17], 1, ctypes.c_void_p(0x10002), 0, None) == \
         ab.ATTN_ERR_INVALID_ARG
+    # relative-position table: R must be in [0, 2^20]
+    assert lib.attn_fwd_score_mod(*args[:17], 2, A, -1, None) == ab.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_score_mod(*args[:17], 2, A, (1 << 20) + 1, None) == \
+        ab.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_score_mod(*args[:17], 2, None, 4, None) == ab.ATTN_ERR_INVALID_ARG
     bad_d = list(args)
     bad_d[10] = 96
     assert lib.attn_fwd_score_mod(*bad_d) == ab.ATTN_ERR_UNSUPPORTED

@@ -68,3 +68,78 @@ def test_zero_slopes_match_plain_forward():
     torch.cuda.synchronize()
     assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
     assert (l1 - l2).abs().max().item() <= 1e-4
+
+
+def rel_table(seed, H, R, spread=1.5):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(H, 2 * R + 1, generator=g) * spread).float()
+
+
+REL_CASES = [
+    # seed, B, Hq, Hkv, Lq, Lk, d, mask, window, bd, doc, R
+    (31, 1, 4, 4, 128, 128, 64, "causal", (-1, -1), 1, False, 16),
+    (32, 2, 8, 2, 300, 300, 64, "causal", (-1, -1), 1, False, 200),   # R past a tile
+    (33, 1, 4, 1, 257, 700, 128, "none", (-1, -1), 1, False, 64),     # both signs of j - p
+    (34, 1, 2, 2, 500, 500, 128, "causal", (100, 0), 1, True, 7),
+    (35, 2, 4, 4, 16, 2064, 128, "draft", (512, 512), 16, True, 32),
+    (36, 1, 8, 8, 1, 3000, 64, "causal", (-1, -1), 1, False, 0),      # per-head constant
+    (37, 1, 2, 2, 640, 640, 64, "none", (-1, -1), 1, False, 1000),    # R beyond every distance
+]
+
+
+@pytest.mark.parametrize("case", REL_CASES,
+                         ids=lambda c: f"s{c[0]}_{c[7]}_lq{c[4]}_lk{c[5]}_d{c[6]}_R{c[11]}")
+def test_relative_bias_matches_oracle(case):
+    seed, B, Hq, Hkv, Lq, Lk, d, mask, window, bd, doc, R = case
+    q, k, v, doc_ids, _ = random_case(seed, B, Hq, Hkv, Lq, Lk, d, doc_split=doc, n_docs=3)
+    table = rel_table(seed, Hq, R)
+    kw = dict(scale=1.0 / math.sqrt(d), mask=mask, window=window, draft_block=bd)
+    qd, kd, vd = to_dev(q, k, v)
+    o, lse = ab.attn_fwd_score_mod(qd, kd, vd, rel_bias=(table.cuda(), R),
+                                   doc_ids=None if doc_ids is None else doc_ids.cuda(), **kw)
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    ro, rl = oracle.attn_fwd(q, k, v, doc_ids=doc_ids, rel_bias=(table.double().numpy(), R),
+                             **kw)
+    compare(o, lse, ro, rl, str(case))
+
+
+@pytest.mark.parametrize("mod", ["alibi", "rel"])
+def test_packed_sequences_with_a_score_modifier(mod):
+    """attn_fwd_varlen_score_mod: each sequence's rows use their own positions."""
+    from workloads import packed_case, packed_lengths
+    H, d = 4, 64
+    lens = packed_lengths(41, 6, 1, 700) + [128, 129]
+    q, k, v, cu_q, cu_k = packed_case(41, lens, lens, H, H, d)
+    kw = {}
+    okw = {}
+    if mod == "alibi":
+        sl = slopes_for(H)
+        kw["alibi_slopes"] = sl.cuda()
+        okw["alibi_slopes"] = sl.double().numpy()
+    else:
+        table = rel_table(42, H, 40)
+        kw["rel_bias"] = (table.cuda(), 40)
+        okw["rel_bias"] = (table.double().numpy(), 40)
+    qd, kd, vd, cqd, ckd = to_dev(q, k, v, cu_q, cu_k)
+    o, lse = ab.attn_fwd_varlen(qd, kd, vd, cqd, ckd, max(lens), mask="causal", **kw)
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    ro, rl = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, mask="causal", **okw)
+    # packed LSE is [H, total]: compare token-major like O
+    compare(o, lse.t(), ro, np.ascontiguousarray(rl.T), f"varlen {mod}")
+
+
+def test_constant_table_matches_plain_forward():
+    """R = 0 with one value per head: the same O, the LSE shifted by the value."""
+    q, k, v, _, _ = random_case(43, 1, 4, 2, 333, 333, 128)
+    qd, kd, vd = to_dev(q, k, v)
+    consts = torch.tensor([[0.5], [-1.0], [2.0], [0.0]], dtype=torch.float32)
+    o1, l1 = ab.attn_fwd_score_mod(qd, kd, vd, rel_bias=(consts.cuda(), 0), mask="causal")
+    o2, l2 = ab.attn_fwd(qd, kd, vd, mask="causal")
+    torch.cuda.synchronize()
+    assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
+    shift = (l1 - l2).cpu()
+    assert (shift - consts.view(1, 4, 1)).abs().max().item() <= 1e-3

@@ -584,7 +584,7 @@ def main():
         workloads = {}
         if not args.no_secondary:
             for sc in (CAUSAL_32K_GQA, DRAFT_WINDOW_DOC, DRAFT_WINDOW_DOC_FULL):
-                c2, _, ms2, fl2, by2 = run_prefill(sc, timer, max(3, args.steps // 20), 3, stream)
+                c2, _, ms2, fl2, by2 = run_prefill(sc, timer, max(10, args.steps // 10), 3, stream)
                 med = statistics.median(ms2)
                 tf = fl2 / (med * 1e9)
                 gbs = by2 / (med * 1e6)

@@ -248,7 +248,8 @@ int attn_decode_num_splits(int B, int Hq, int Hkv, int Lq, int Lk_max, int d, in
  *   offset 0:           fp32 O_s  [nsplit, B*Hq*Lq, d]   (normalised per split)
  *   offset ws_lse_off:  fp32 LSE_s [nsplit, B*Hq*Lq]
  *   where ws_lse_off = round_up(nsplit*B*Hq*Lq*d*4, 256).
- *   Rows of splits that hold no key of their sequence are not written.
+ *   Splits that hold no key of their sequence write LSE_s = -inf for their
+ *   rows and leave O_s unwritten; the combine gives them weight 0.
  */
 size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk_max, int d,
                                   int num_splits);

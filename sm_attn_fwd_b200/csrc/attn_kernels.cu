@@ -23,6 +23,10 @@
 //               over S_j in TMEM, and finally stores O / l and the LSE.
 // Tensor memory: S double buffer at columns [0,128) and [128,256), O at
 // [256, 256 + d).  Key tiles that the mask empties entirely are never loaded.
+// A paged cache whose pages are shorter than a key tile takes one TMA box per
+// page and 64-column atom (16 per K tile for 16-key pages at d = 128); the
+// boxes of a tile are then issued by three copy warps (warps 0, 6 and 7), as
+// one issuing warp bounds the stream.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -39,7 +43,10 @@ __device__ int g_device_error = 0;
 
 namespace {
 
-constexpr int kThreads = 192;
+// warps 0 (producer), 1 (MMA), 2..5 (softmax), 6..7 (extra copy warps for
+// pages shorter than a key tile)
+constexpr int kThreads = 256;
+constexpr int kCopyWarps = 3;
 constexpr int kTmemCols = 512;
 constexpr uint32_t kTmemO = 256;
 // S (and P over it) double buffer: columns [0,128) and [128,256).
@@ -140,16 +147,27 @@ __global__ void __launch_bounds__(kThreads, 1)
     kv_len = kv_len < 0 ? 0 : p.Lk;
   }
   const int c0 = split * p.chunk;
-  if (c0 >= kv_len) return;  // this split holds no keys of sequence b (uniform exit)
-  const int key_end = min(c0 + p.chunk, kv_len);  // keys at or past this are never visible
   const int rows_valid = min(kBlockM, p.group * p.Lq - rt * kBlockM);
   // flat output row of tile row 0
   const long long row_out0 =
       ((long long)b * p.Hq + (long long)hkv * p.group) * p.Lq + (long long)rt * kBlockM;
+  if (c0 >= kv_len) {
+    // This split holds no keys of sequence b: its rows get LSE = -inf, which
+    // the combine reads as weight 0 (their O rows are never written or read).
+    if ((int)threadIdx.x < rows_valid)
+      p.ws_lse[(long long)split * p.B * p.Hq * p.Lq + row_out0 + threadIdx.x] = -INFINITY;
+    return;  // uniform exit
+  }
+  const int key_end = min(c0 + p.chunk, kv_len);  // keys at or past this are never visible
   const int q_coord_y = (int)row_out0;
   const int kv_z = b * p.Hkv + hkv;
   const int t_lo = c0 / kBlockN;  // candidate key tiles (absolute tile indices)
   const int t_hi = (key_end - 1) / kBlockN;
+  // pages shorter than a key tile: three copy warps share the TMA boxes of
+  // every K/V tile (one box per page slice and atom; a single issuing warp
+  // bounds the stream there)
+  const bool small_pages = p.block_table != nullptr && p.page_size < kBlockN;
+  const uint32_t kv_arrivals = small_pages ? kCopyWarps : 1u;
 
   // ------------------------------------------------------------- prologue
   if (warp == 0) {
@@ -159,9 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tm_v);
       ptx::mbar_init(q_full, 1);
       for (int s = 0; s < C::kStages; ++s) {
-        ptx::mbar_init(&k_full[s], 1);
+        ptx::mbar_init(&k_full[s], kv_arrivals);
         ptx::mbar_init(&k_empty[s], 1);
-        ptx::mbar_init(&v_full[s], 1);
+        ptx::mbar_init(&v_full[s], kv_arrivals);
         ptx::mbar_init(&v_empty[s], 1);
       }
       for (int s = 0; s < 2; ++s) {
@@ -203,25 +221,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = misc->tmem_base;
   const int n_tiles = misc->n_tiles;
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
-    // The whole warp runs this loop; lane 0 owns the barrier bookkeeping and the
-    // lanes share out the TMA boxes of a tile (many boxes for small pages).
+  if (warp == 0 || (warp >= 6 && small_pages)) {
+    // ------------------------------------------------------------ producer
+    // Copy warp cw (warp 0, and warps 6 and 7 when pages are shorter than a
+    // key tile) issues its share of the TMA boxes of every K and V tile and
+    // arrives once per tile on k_full / v_full with the bytes of its own
+    // boxes; lane 0 of warp 0 also loads Q.
+    const int cw = warp == 0 ? 0 : warp - 5;
     if (n_tiles > 0) {
       constexpr uint32_t kTx = C::kTileBytes;
-      if (lane == 0) {
+      if (warp == 0 && lane == 0) {
         ptx::mbar_arrive_expect_tx(q_full, kTx);
         for (int a = 0; a < C::kAtoms; ++a)
           ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, q_coord_y);
       }
-      // One 128-key K or V tile into shared memory.  Contiguous cache: one box
-      // per 64-column atom.  Paged cache ([num_pages, Hkv, page_size, d] through
-      // the block table): pages of 128 keys or more give one box per atom at
-      // the key's offset inside its page; smaller pages give one box per page
-      // slice, each landing on a whole number of 8-row swizzle atoms, so the
-      // assembled tile is laid out exactly like a single box.  Keys past the
-      // block table read as zeros (out-of-range coordinate), as do pages whose
-      // id is out of range (which also flags the device error word).
+      // Contiguous cache: one box per 64-column atom.  Paged cache
+      // ([num_pages, Hkv, page_size, d] through the block table): pages of 128
+      // keys or more give one box per atom at the key's offset inside its
+      // page; smaller pages give one box per page slice, each landing on a
+      // whole number of 8-row swizzle atoms, so the assembled tile is laid out
+      // exactly like a single box.  Keys past the block table read as zeros
+      // (out-of-range coordinate), as do pages whose id is out of range (which
+      // also flags the device error word).
       auto page_z = [&](int key) -> int {
         const int idx = key / p.page_size;
         if (idx >= p.pages_per_seq) return -1;
@@ -232,37 +253,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return page * p.Hkv + hkv;
       };
-      auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int k0) {
-        if (p.block_table == nullptr) {
-          if (lane < C::kAtoms)
-            ptx::tma_load_3d(dst + lane * C::kAtomBytes, tm, bar, lane * 64, k0, kv_z);
-        } else if (p.page_size >= kBlockN) {
-          if (lane < C::kAtoms)
-            ptx::tma_load_3d(dst + lane * C::kAtomBytes, tm, bar, lane * 64, k0 % p.page_size,
-                             page_z(k0));
+      // This warp's boxes of one K or V tile, with its own expect-tx.  Small
+      // pages: lane i < `mine` loads item cw + kCopyWarps * i (page slice
+      // item / atoms, atom item % atoms) from pool index pz (its page, fetched
+      // one tile ahead).
+      const int n_items = small_pages ? (kBlockN / p.page_size) * C::kAtoms : 0;
+      const int mine = small_pages ? (n_items - cw + kCopyWarps - 1) / kCopyWarps : 0;
+      const int item = cw + kCopyWarps * lane;
+      auto item_page = [&](int t) -> int {
+        if (!small_pages) return lane < C::kAtoms ? page_z(t * kBlockN) : -1;
+        return lane < mine ? page_z(t * kBlockN + (item / C::kAtoms) * p.page_size) : -1;
+      };
+      auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int k0, int pz) {
+        if (!small_pages) {
+          if (lane == 0) ptx::mbar_arrive_expect_tx(bar, kTx);
+          __syncwarp();
+          if (lane < C::kAtoms) {
+            const int y = p.block_table == nullptr ? k0 : k0 % p.page_size;
+            const int z = p.block_table == nullptr ? kv_z : pz;
+            ptx::tma_load_3d(dst + lane * C::kAtomBytes, tm, bar, lane * 64, y, z);
+          }
         } else {
-          const int n_items = (kBlockN / p.page_size) * C::kAtoms;
-          for (int item = lane; item < n_items; item += 32) {
+          if (lane == 0) ptx::mbar_arrive_expect_tx(bar, (uint32_t)(mine * p.page_size * 128));
+          __syncwarp();
+          if (lane < mine) {
             const int sub = item / C::kAtoms, a = item % C::kAtoms;
             ptx::tma_load_3d(dst + a * C::kAtomBytes + sub * p.page_size * 128, tm, bar, a * 64,
-                             0, page_z(k0 + sub * p.page_size));
+                             0, pz);
           }
         }
       };
       int j = 0;
       bool ok = true;
+      const bool paged = p.block_table != nullptr;
+      int pz_next = paged ? item_page(t_lo) : 0;
       for (int t = t_lo; t <= t_hi && ok; ++t) {
         if (bit_get(empty_bits, t - t_lo)) continue;
         const int s = j % C::kStages;
         const uint32_t ph = (uint32_t)(j / C::kStages) & 1u;
         const int k0 = t * kBlockN;
+        const int pz = pz_next;
         ok = ptx::mbar_wait(&k_empty[s], ph ^ 1u, abort_flag, &g_device_error,
                             kDevErrTimeoutProducer);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        if (lane == 0) ptx::mbar_arrive_expect_tx(&k_full[s], kTx);
-        __syncwarp();
-        load_kv(sK + s * C::kTileBytes, &tm_k, &k_full[s], k0);
+        load_kv(sK + s * C::kTileBytes, &tm_k, &k_full[s], k0, pz);
+        if (paged && t < t_hi) pz_next = item_page(t + 1);  // in flight during the wait
         ok = ptx::mbar_wait(&v_empty[s], ph ^ 1u, abort_flag, &g_device_error,
                             kDevErrTimeoutProducer);
         ok = __all_sync(0xffffffffu, ok);
@@ -270,14 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++j;  // the K load of this tile is in flight; drain it below
           break;
         }
-        if (lane == 0) ptx::mbar_arrive_expect_tx(&v_full[s], kTx);
-        __syncwarp();
-        load_kv(sV + s * C::kTileBytes, &tm_v, &v_full[s], k0);
+        load_kv(sV + s * C::kTileBytes, &tm_v, &v_full[s], k0, pz);
         ++j;
       }
-      // Drain: every TMA write into shared memory must land before the CTA exits.
-      // In a normal run these phases have completed already.
-      if (lane == 0) {
+      // Drain: every write into shared memory lands before the CTA exits (in a
+      // normal run these phases have completed already).  The phases of
+      // k_full / v_full cover every copy warp's loads.
+      if (warp == 0 && lane == 0) {
         int dummy_abort = 0;
         ptx::mbar_wait(q_full, 0, &dummy_abort, nullptr, 0);
         for (int jj = max(0, j - C::kStages); jj < j; ++jj) {
@@ -347,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int dummy_abort = 0;
       ptx::mbar_wait(mma_drain, 0, &dummy_abort, nullptr, 0);
     }
-  } else {
+  } else if (warp >= 2 && warp < 6) {
     // ----------------------------------------------------------- softmax
     const int quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;      // tile row == TMEM lane
@@ -510,52 +545,77 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Split-KV combine (the LSE-weighted merge of FlashDecoding-style partials):
 //   LSE = log sum_s exp(LSE_s),  O = sum_s exp(LSE_s - LSE) O_s.
-// One warp per output row; lane i owns d/32 consecutive elements.
+// One warp per output row; lane i owns d/32 consecutive elements.  The split
+// LSEs are read one per lane (32 splits per load), and the partial rows of
+// kUnroll splits are loaded together: a row costs two memory round trips (the
+// LSEs, then the partial rows), not two per split.
 template <int D>
 __global__ void __launch_bounds__(256) attn_decode_combine_kernel(const FwdParams p) {
   constexpr int kPer = D / 32;
+  constexpr int kUnroll = 8;
   constexpr float kLog2e = 1.44269504088896340736f;
   const long long nrows = (long long)p.B * p.Hq * p.Lq;
   const long long row = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
-  if (row >= nrows) return;
-  const int b = (int)(row / ((long long)p.Hq * p.Lq));
-  int kv_len = p.kv_lens[b];
-  kv_len = kv_len < 0 ? 0 : (kv_len > p.Lk ? p.Lk : kv_len);
-  const int ns = (kv_len + p.chunk - 1) / p.chunk;
+  if (row >= nrows) return;  // warp-uniform
+  // every split wrote this row's LSE (-inf where it held no key of the sequence)
+  const int ns = p.nsplit;
   float mx = -INFINITY;
-  for (int s = 0; s < ns; ++s) mx = fmaxf(mx, p.ws_lse[(long long)s * nrows + row]);
+  for (int s0 = 0; s0 < ns; s0 += 32) {
+    if (s0 + lane < ns) mx = fmaxf(mx, p.ws_lse[(long long)(s0 + lane) * nrows + row]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   float acc[kPer];
 #pragma unroll
   for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
   float sum = 0.0f;
   if (mx != -INFINITY) {
-    for (int s = 0; s < ns; ++s) {
-      const float ls = p.ws_lse[(long long)s * nrows + row];
-      if (ls == -INFINITY) continue;
-      const float w = ptx::ex2((ls - mx) * kLog2e);
-      sum += w;
-      const float* src = p.ws_o + ((long long)s * nrows + row) * D + lane * kPer;
-      if constexpr (kPer == 4) {
-        const float4 v = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
-        acc[2] += w * v.z;
-        acc[3] += w * v.w;
-      } else {
-        const float2 v = *reinterpret_cast<const float2*>(src);
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
+    for (int s0 = 0; s0 < ns; s0 += 32) {
+      // lane i: weight of split s0 + i (0 for a split with no visible key)
+      const float ls = s0 + lane < ns ? p.ws_lse[(long long)(s0 + lane) * nrows + row] : -INFINITY;
+      const float w_lane = ls == -INFINITY ? 0.0f : ptx::ex2((ls - mx) * kLog2e);
+      sum += w_lane;
+      const int n = min(32, ns - s0);
+      for (int i0 = 0; i0 < n; i0 += kUnroll) {
+        float wv[kUnroll];
+        float v[kUnroll][kPer];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          wv[u] = __shfl_sync(0xffffffffu, w_lane, (i0 + u) & 31);
+          const bool use = i0 + u < n && wv[u] != 0.0f;
+          const float* src =
+              p.ws_o + ((long long)(s0 + i0 + u) * nrows + row) * D + lane * kPer;
+          if constexpr (kPer == 4) {
+            const float4 t = use ? *reinterpret_cast<const float4*>(src)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            v[u][0] = t.x;
+            v[u][1] = t.y;
+            v[u][2] = t.z;
+            v[u][3] = t.w;
+          } else {
+            const float2 t = use ? *reinterpret_cast<const float2*>(src) : make_float2(0.f, 0.f);
+            v[u][0] = t.x;
+            v[u][1] = t.y;
+          }
+          if (!use) wv[u] = 0.0f;
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+#pragma unroll
+          for (int i = 0; i < kPer; ++i) acc[i] += wv[u] * v[u][i];
       }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
   }
   const float inv = sum > 0.0f ? 1.0f / sum : 0.0f;
   __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.o) + row * D + lane * kPer;
   if constexpr (kPer == 4) {
-    uint2 v;
-    v.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    v.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(dst) = v;
+    uint2 o2;
+    o2.x = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    o2.y = ptx::pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = o2;
   } else {
     *reinterpret_cast<uint32_t*>(dst) = ptx::pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }

@@ -12,9 +12,11 @@
 // B200 mapping.  A work unit is two adjacent 128-row query tiles (A and B) of
 // one (batch, head); both consume the same K/V tiles, so one TMA stream feeds
 // four tcgen05 MMAs per key tile (S_A, S_B, P_A V, P_B V).  384 threads:
-//   warpgroup 0   warp 0: builds each unit's tile schedule (EMPTY / PARTIAL /
+//   warpgroup 0   warp 3: builds each unit's tile schedule (EMPTY / PARTIAL /
 //                 FULL per key tile and query tile, in shared memory, double
-//                 buffered) and issues the TMA loads (Q_A, Q_B, K/V ring);
+//                 buffered), one unit ahead of the others, so the document-id
+//                 loads of the classification never hold up the loads;
+//                 warp 0: issues the TMA loads (Q_A, Q_B, K/V ring);
 //                 warp 1 (and warp 2 for d = 64, one per query tile):
 //                 allocate tensor memory and issue every MMA (elect.sync picks
 //                 the issuing lane); registers lowered to 80 per thread.
@@ -97,8 +99,8 @@ enum : int {
   kPFull = 6,        // [2] softmax x (128 arrivals) -> MMA: P_x written, O_x rescaled
   kODone = 8,        // [2] MMA -> softmax x: P_x V done
   kOFree = 10,       // [2] softmax x (128) -> MMA: O_x read out, may be overwritten
-  kSchedFull = 12,   // [2] schedule builder -> MMA, softmax
-  kSchedEmpty = 14,  // [2] MMA + 8 softmax warps -> schedule builder
+  kSchedFull = 12,   // [2] schedule builder -> TMA, MMA, softmax
+  kSchedEmpty = 14,  // [2] TMA + MMA + 8 softmax warps -> schedule builder
   kDrain = 16,       // MMA: all MMAs done
   kSFree = 17,       // [2] softmax x (128) -> MMA: S_x loaded into registers (separate-P mode)
   kTurn = 19,        // [2] softmax 1-x (128) -> softmax x: x may run its exponentials
@@ -160,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&bars[kODone + x], 1);
       ptx::mbar_init(&bars[kOFree + x], 128);
       ptx::mbar_init(&bars[kSchedFull + x], 1);
-      ptx::mbar_init(&bars[kSchedEmpty + x], kMmaWarps + 8);
+      ptx::mbar_init(&bars[kSchedEmpty + x], 1 + kMmaWarps + 8);
       ptx::mbar_init(&bars[kSFree + x], 128);
       ptx::mbar_init(&bars[kTurn + x], 128);
     }
@@ -189,8 +191,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 4) {
     ptx::regs_dec<kRegsLow>();
-    if (warp == 0) {
-      // ---------------------------------------- schedule builder + TMA producer
+    if (warp == 3) {
+      // -------------------------------------------------- schedule builder
+      for (int r = 0;; ++r) {
+        const int u = unit_of(p, cta, r);
+        if (u < 0) break;
+        Unit w;
+        decode_unit(p, u, w);
+        if (w.bad && lane == 0) atomicOr(err, kDevErrBadSeqlens);
+        bool ok = ptx::mbar_wait_a(BAR(kSchedEmpty + (r & 1)), (((uint32_t)r >> 1) & 1u) ^ 1u,
+                                   abort_flag, err, kDevErrTimeoutProducer);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        build_sched(p, w, &scheds[r & 1], lane);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_a(BAR(kSchedFull + (r & 1)));
+      }
+    } else if (warp == 0) {
+      // ---------------------------------------------------------- TMA producer
       int jkv = 0;
       int rounds = 0;
       bool ok = true;
@@ -200,16 +218,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         rounds = r + 1;
         Unit w;
         decode_unit(p, u, w);
-        if (w.bad && lane == 0) atomicOr(err, kDevErrBadSeqlens);
-        Sched* s = &scheds[r & 1];
-        ok = ptx::mbar_wait_a(BAR(kSchedEmpty + (r & 1)), (((uint32_t)r >> 1) & 1u) ^ 1u,
-                              abort_flag, err, kDevErrTimeoutProducer);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        build_sched(p, w, s, lane);
-        __syncwarp();
+        const Sched* s = &scheds[r & 1];
         if (lane == 0) {
-          ptx::mbar_arrive_a(BAR(kSchedFull + (r & 1)));
+          ok = ptx::mbar_wait_a(BAR(kSchedFull + (r & 1)), ((uint32_t)r >> 1) & 1u, abort_flag,
+                                err, kDevErrTimeoutProducer);
           constexpr uint32_t kTx = C::kTileBytes;
           for (int x = 0; x < 2 && ok; ++x) {
             ok = ptx::mbar_wait_a(BAR(kQEmpty + x), ((uint32_t)r & 1u) ^ 1u, abort_flag, err,
@@ -253,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  packed ? w.k_base + t * 128 : kv_z);
             ++jkv;
           }
+          ptx::mbar_arrive_a(BAR(kSchedEmpty + (r & 1)));  // done reading the schedule
         }
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
         jkv = __shfl_sync(0xffffffffu, jkv, 0);

@@ -171,17 +171,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(mma_drain, 1);
       misc->abort = 0;
       ptx::fence_mbar_init();
+      // Q does not depend on the classification below: its load starts now
+      ptx::mbar_arrive_expect_tx(q_full, C::kTileBytes);
+      for (int a = 0; a < C::kAtoms; ++a)
+        ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, (int)row_out0);
     }
     // Tile classification over the valid rows: the union [u_lo, u_hi] of their
     // key intervals decides EMPTY, the intersection [i_lo, i_hi] FULL; with
     // document ids a tile whose documents miss every row's document is EMPTY,
     // and FULL needs one document shared by the whole tile and every row.
     long long u_lo = 0x7fffffffffffLL, u_hi = -1, i_lo = 0, i_hi = 0x7fffffffffffLL;
-    int qdmin = 0x7fffffff, qdmax = (int)0x80000000;
     for (int r = lane; r < rows_valid; r += 32) {
       long long lo, hi;
-      const long long pos = row_pos(r);
-      prefill::key_bounds(p, p.Lk, pos, lo, hi);
+      prefill::key_bounds(p, p.Lk, row_pos(r), lo, hi);
       lo = max(lo, 0LL);
       if (hi >= lo) {
         u_lo = min(u_lo, lo);
@@ -189,20 +191,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       i_lo = max(i_lo, lo);
       i_hi = min(i_hi, hi);
-      if (doc_b != nullptr && pos >= 0) {
-        const int d = __ldg(doc_b + pos);
-        qdmin = min(qdmin, d);
-        qdmax = max(qdmax, d);
-      }
     }
     for (int o = 16; o > 0; o >>= 1) {
       u_lo = min(u_lo, __shfl_xor_sync(0xffffffffu, u_lo, o));
       u_hi = max(u_hi, __shfl_xor_sync(0xffffffffu, u_hi, o));
       i_lo = max(i_lo, __shfl_xor_sync(0xffffffffu, i_lo, o));
       i_hi = min(i_hi, __shfl_xor_sync(0xffffffffu, i_hi, o));
-      qdmin = min(qdmin, __shfl_xor_sync(0xffffffffu, qdmin, o));
-      qdmax = max(qdmax, __shfl_xor_sync(0xffffffffu, qdmax, o));
     }
+    // document ids: Lq <= Lk, so every row position is a key index
+    int qdmin = 0x7fffffff, qdmax = (int)0x80000000;
+    if (doc_b != nullptr) prefill::doc_range_rows(doc_b, rows_valid, lane, row_pos, qdmin, qdmax);
     const int ntc = t_hi - t_lo + 1;
     int n_tiles = 0;
     for (int base = 0; base < ntc; base += 32) {
@@ -211,22 +209,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool empty = i >= ntc || u_hi < 0 || k0 > u_hi || k0 + kBlockN - 1 < u_lo;
       bool full = !empty && (k0 + kBlockN <= p.Lk) && i_lo <= k0 && i_hi >= k0 + kBlockN - 1;
       if (doc_b != nullptr) {
-        for (int ww = 0; ww < 32 && base + ww < ntc; ++ww) {
-          const long long kb = (long long)(t_lo + base + ww) * kBlockN;
-          const int kend = (int)min(kb + kBlockN, (long long)p.Lk);
-          int mn = 0x7fffffff, mx = (int)0x80000000;
-          for (long long kk = kb + lane; kk < kend; kk += 32) {
-            const int d = __ldg(doc_b + kk);
-            mn = min(mn, d);
-            mx = max(mx, d);
-          }
-          for (int o = 16; o > 0; o >>= 1) {
-            mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          }
-          if (lane == ww) {
-            if (mx < qdmin || mn > qdmax) empty = true;
-            if (!(mn == mx && qdmin == qdmax && mn == qdmin)) full = false;
+        constexpr int kBatch = 4;
+        for (int ww0 = 0; ww0 < 32 && base + ww0 < ntc; ww0 += kBatch) {
+          int mn[kBatch], mx[kBatch];
+          prefill::doc_range_tiles<kBlockN, kBatch>(doc_b, p.Lk, t_lo + base + ww0, t_lo + ntc,
+                                                    lane, mn, mx);
+#pragma unroll
+          for (int u = 0; u < kBatch; ++u) {
+            if (lane == ww0 + u) {
+              if (mx[u] < qdmin || mn[u] > qdmax) empty = true;
+              if (!(mn[u] == mx[u] && qdmin == qdmax && mn[u] == qdmin)) full = false;
+            }
           }
         }
       }
@@ -253,9 +246,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------ TMA producer
     if (n_tiles > 0 && lane == 0) {
       constexpr uint32_t kTx = C::kTileBytes;
-      ptx::mbar_arrive_expect_tx(q_full, kTx);
-      for (int a = 0; a < C::kAtoms; ++a)
-        ptx::tma_load_2d(sQ + a * C::kAtomBytes, &tm_q, q_full, a * 64, (int)row_out0);
       int j = 0;
       bool ok = true;
       for (int t = t_lo; t <= t_hi && ok; ++t) {
@@ -285,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // Drain: every TMA write into shared memory lands before the partials
       // reuse the ring (in a normal run these phases completed long ago).
       int dummy_abort = 0;
-      ptx::mbar_wait(q_full, 0, &dummy_abort, nullptr, 0);
       for (int jj = max(0, j - C::kStages); jj < j; ++jj) {
         const int s = jj % C::kStages;
         const uint32_t ph = (uint32_t)(jj / C::kStages) & 1u;
@@ -294,6 +283,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         dummy_abort = 0;
         ptx::mbar_wait(&v_full[s], ph, &dummy_abort, nullptr, 0);
       }
+    }
+    if (lane == 0) {  // the Q load was issued in the prologue, whatever n_tiles is
+      int dummy_abort = 0;
+      ptx::mbar_wait(q_full, 0, &dummy_abort, nullptr, 0);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------- MMA issuer

@@ -1,7 +1,8 @@
-// Device helpers shared by the two prefill kernels (attn_prefill.cu for head
-// dimension 128, attn_prefill64.cu for 64): the work-unit numbering, the
-// per-row visible key interval of the mask predicate, and the per-unit tile
-// schedule (EMPTY / PARTIAL / FULL per key tile and query tile).
+// Device helpers shared by the prefill kernels (the persistent kernel in
+// attn_prefill.cu and the short-query kernel in attn_short.cu): the work-unit
+// numbering, the per-row visible key interval of the mask predicate, the
+// document ranges of rows and key tiles, and the per-unit tile schedule
+// (EMPTY / PARTIAL / FULL per key tile and query tile).
 //
 // Masks: the mask_mod predicate of "FlexAttention 是什么，以及 DFlash2 之谜的完整
 // 侦破" (section 1: causal, sliding window, non-causal, document ids; section 3:
@@ -98,6 +99,86 @@ __device__ __forceinline__ int unit_of(const FwdParams& p, int cta, int r) {
   return idx < p.n_units ? idx : -1;
 }
 
+__device__ __forceinline__ void warp_min_max(int& mn, int& mx) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+}
+
+// Whole warp: [mn, mx] of the document ids doc_b[pos(r)] of rows r < rows
+// (rows <= 128).  All four loads of a lane are issued before any is used, so
+// the warp pays one memory round trip, not one per 32 rows.  An empty range
+// gives mn = INT_MAX, mx = INT_MIN.
+template <typename PosFn>
+__device__ __forceinline__ void doc_range_rows(const int32_t* doc_b, int rows, int lane, PosFn pos,
+                                               int& mn, int& mx) {
+  int d[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int r = lane + 32 * m;
+    d[m] = r < rows ? __ldg(doc_b + pos(r)) : 0;
+  }
+  mn = 0x7fffffff;
+  mx = (int)0x80000000;
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    if (lane + 32 * m < rows) {
+      mn = min(mn, d[m]);
+      mx = max(mx, d[m]);
+    }
+  }
+  warp_min_max(mn, mx);
+}
+
+// Whole warp: document range [mn[u], mx[u]] of key tiles t0 + u, u < kBatch,
+// of kBN keys each (keys at or past Lk and tiles at or past t_end ignored).
+// The kBatch * kBN / 32 loads of a lane are all in flight together; when the
+// whole batch lies inside [0, Lk) and before t_end they come from one base
+// address with constant offsets and need no predicates.
+template <int kBN, int kBatch>
+__device__ __forceinline__ void doc_range_tiles(const int32_t* doc_b, int Lk, int t0, int t_end,
+                                                int lane, int (&mn)[kBatch], int (&mx)[kBatch]) {
+  constexpr int kPer = kBN / 32;
+  const long long k_first = (long long)t0 * kBN;
+  const int32_t* base = doc_b + k_first + lane;
+  if (t0 + kBatch <= t_end && k_first + kBatch * kBN <= Lk) {
+    int d[kBatch][kPer];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+      for (int m = 0; m < kPer; ++m) d[u][m] = __ldg(base + u * kBN + 32 * m);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      mn[u] = mx[u] = d[u][0];
+#pragma unroll
+      for (int m = 1; m < kPer; ++m) {
+        mn[u] = min(mn[u], d[u][m]);
+        mx[u] = max(mx[u], d[u][m]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      mn[u] = 0x7fffffff;
+      mx[u] = (int)0x80000000;
+      if (t0 + u < t_end) {
+#pragma unroll
+        for (int m = 0; m < kPer; ++m) {
+          if (k_first + u * kBN + lane + 32 * m < Lk) {
+            const int d = __ldg(base + u * kBN + 32 * m);
+            mn[u] = min(mn[u], d);
+            mx[u] = max(mx[u], d);
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) warp_min_max(mn[u], mx[u]);
+}
+
 // Tile schedule of one unit for key tiles of kBN keys: bit i of empty[x] /
 // full[x] describes key tile t_lo + i for query tile x.
 template <int kBN>
@@ -145,18 +226,8 @@ __device__ void build_sched(const FwdParams& p, const Unit& w, Sched<kBN>* s, in
   if (doc_b) {
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
-      int mn = 0x7fffffff, mx = (int)0x80000000;
-      for (int r = lane; r < w.rows[x]; r += 32) {
-        const int d = __ldg(doc_b + (w.pos0[x] + r));
-        mn = min(mn, d);
-        mx = max(mx, d);
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      }
-      qdmin[x] = mn;
-      qdmax[x] = mx;
+      const long long p0 = w.pos0[x];
+      doc_range_rows(doc_b, w.rows[x], lane, [&](int r) { return p0 + r; }, qdmin[x], qdmax[x]);
     }
   }
   int cnt[2] = {0, 0}, last[2] = {-1, -1};
@@ -171,24 +242,18 @@ __device__ void build_sched(const FwdParams& p, const Unit& w, Sched<kBN>* s, in
                 (hi_first[x] >= k0 + kBN - 1);
     }
     if (doc_b) {
-      for (int ww = 0; ww < 32 && base + ww < ntc; ++ww) {
-        const long long kb = (long long)(t_lo + base + ww) * kBN;
-        const int kend = (int)min(kb + kBN, (long long)p.Lk);
-        int mn = 0x7fffffff, mx = (int)0x80000000;
-        for (long long kk = kb + lane; kk < kend; kk += 32) {
-          const int d = __ldg(doc_b + kk);
-          mn = min(mn, d);
-          mx = max(mx, d);
-        }
-        for (int o = 16; o > 0; o >>= 1) {
-          mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-          mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-        }
-        if (lane == ww) {
+      constexpr int kBatch = 4;
+      for (int ww0 = 0; ww0 < 32 && base + ww0 < ntc; ww0 += kBatch) {
+        int mn[kBatch], mx[kBatch];
+        doc_range_tiles<kBN, kBatch>(doc_b, p.Lk, t_lo + base + ww0, t_lo + ntc, lane, mn, mx);
 #pragma unroll
-          for (int x = 0; x < 2; ++x) {
-            if (mx < qdmin[x] || mn > qdmax[x]) empty[x] = true;
-            if (!(mn == mx && qdmin[x] == qdmax[x] && mn == qdmin[x])) full[x] = false;
+        for (int u = 0; u < kBatch; ++u) {
+          if (lane == ww0 + u) {
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+              if (mx[u] < qdmin[x] || mn[u] > qdmax[x]) empty[x] = true;
+              if (!(mn[u] == mx[u] && qdmin[x] == qdmax[x] && mn[u] == qdmin[x])) full[x] = false;
+            }
           }
         }
       }

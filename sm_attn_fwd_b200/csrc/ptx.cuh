@@ -213,17 +213,6 @@ __device__ __forceinline__ void mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
-__device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 __device__ __forceinline__ void mma_commit_warp(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -257,26 +246,6 @@ __device__ __forceinline__ void mma_pv_chain8(uint32_t d_tmem, uint32_t a_tmem, 
       "add.u32 a, %1, 48;  add.s64 b, %2, 768;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t"
       "add.u32 a, %1, 56;  add.s64 b, %2, 896;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-//   O (+)= P V over 64 keys: 4 MMAs, A = P in TMEM (8 columns per step),
-//   B = V in shared memory (descriptor start address + 2048 bytes per step).
-__device__ __forceinline__ void mma_pv_chain4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred e, p, one;\n\t.reg .b64 b;\n\t.reg .b32 a;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "setp.eq.u32 one, 0, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
-      "add.u32 a, %1, 8;   add.s64 b, %2, 128;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t"
-      "add.u32 a, %1, 16;  add.s64 b, %2, 256;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t"
-      "add.u32 a, %1, 24;  add.s64 b, %2, 384;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], b, %3, one;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
@@ -406,23 +375,6 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
-// Named barrier `id` over 256 threads that also ORs a flag across them: every
-// participant gets true if any of them passed bad = true.  All participants
-// must reach the same sequence of meetings (there is no timeout here: the
-// callers keep their meeting counts equal on every path, aborts included).
-__device__ __forceinline__ bool pair_meet_any(int id, bool bad) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred b, a;\n\t"
-      "setp.ne.u32 b, %1, 0;\n\t"
-      "bar.red.or.pred a, %2, 256, b;\n\t"
-      "selp.u32 %0, 1, 0, a;\n\t}"
-      : "=r"(out)
-      : "r"((uint32_t)bad), "r"(id)
-      : "memory");
-  return out != 0;
-}
-
 // ------------------------------------------------------------------ clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
@@ -509,12 +461,6 @@ __device__ __forceinline__ void add2_acc(float& s0, float& s1, float a0, float a
       "mov.b64 {%0, %1}, rs;\n\t}"
       : "+f"(s0), "+f"(s1)
       : "f"(a0), "f"(a1));
-}
-// max of three
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
 }
 
 // Maximum of 128 values: sixteen independent chains of two-input max, then a tree.

@@ -88,9 +88,13 @@ def test_decode_split_plan_and_workspace_arithmetic():
     assert (n, chunk.value) == (3, 384)
     n = lib.attn_decode_num_splits(2, 16, 2, 1, 1000, 128, 100, ctypes.byref(chunk))
     assert (n, chunk.value) == (8, 128)           # capped at ceil(1000 / 128)
-    # library choice: chunks never exceed 4096 keys and cover Lk_max
+    # library choice: chunks never exceed 8192 keys and cover Lk_max
     n = lib.attn_decode_num_splits(64, 64, 8, 1, 32768, 128, 0, ctypes.byref(chunk))
-    assert chunk.value <= 4096 and chunk.value % 128 == 0 and n * chunk.value >= 32768
+    assert chunk.value <= 8192 and chunk.value % 128 == 0 and n * chunk.value >= 32768
+    assert (n, chunk.value) == (4, 8192)
+    # few (b, kv head) units: at least two waves of CTAs over the SMs
+    n = lib.attn_decode_num_splits(1, 8, 1, 1, 32768, 128, 0, ctypes.byref(chunk))
+    assert n * 1 >= 2 * 148 or chunk.value == 128
     ws = lib.attn_decode_workspace_size(2, 16, 2, 1, 1000, 128, 3)
     nrows = 2 * 16 * 1
     o_bytes = 3 * nrows * 128 * 4

@@ -62,9 +62,13 @@ def test_paged_decode_matches_gathered_oracle(case):
     compare(o, lse, ro, rl, str(case))
 
 
-def test_paged_equals_contiguous_entry_point():
-    """Identity page table: the paged call and attn_decode_splitkv agree to the bit."""
-    B, Hq, Hkv, Lq, P, pps, d = 2, 16, 2, 1, 128, 8, 128
+@pytest.mark.parametrize("P,d", [(128, 128), (32, 128), (16, 128), (16, 64)])
+def test_paged_equals_contiguous_entry_point(P, d):
+    """Identity page table: the paged call and attn_decode_splitkv agree to the bit
+    (pages shorter than a key tile are copied by the producer lanes, pages of 128
+    by TMA; both must leave the same tile layout in shared memory)."""
+    B, Hq, Hkv, Lq = 2, 16, 2, 1
+    pps = 1024 // P
     g = torch.Generator().manual_seed(9)
     q = torch.randn(B, Hq, Lq, d, generator=g).to(torch.bfloat16)
     k = torch.randn(B, Hkv, pps * P, d, generator=g).to(torch.bfloat16)

@@ -187,6 +187,34 @@ attn_status_t attn_fwd_varlen_score_mod(const void* q, const void* k, const void
                                         void* stream);
 
 /*
+ * attn_fwd_host — attn_fwd on tensors that live in host memory: the same
+ * operation and layouts, with q, k, v, doc_ids (nullable) read from host
+ * buffers and o, lse written to host buffers.
+ *
+ * The call copies the inputs into `workspace` (device memory, owned by the
+ * caller, at least attn_fwd_host_workspace_size bytes, 256-byte aligned), runs
+ * the forward and copies O and the LSE back, all queued on `stream`: read the
+ * outputs after synchronising it.  The work is cut into chunks of whole
+ * (batch, kv head) pairs, and chunk c's uploads, chunk c - 1's kernel and
+ * chunk c - 2's downloads run at the same time (two internal copy streams per
+ * device and context, joined to `stream` by events).  Page-locked (pinned)
+ * host buffers are needed for the copies to overlap; pageable ones work but
+ * serialise.  The chunks use the kernel a single attn_fwd call on the whole
+ * shape would use, so O and LSE are the same bits as attn_fwd's.
+ *
+ * Errors: as attn_fwd (checked before anything is queued); WORKSPACE for a
+ * missing, misaligned or too small workspace.  Enqueueing is serialised across
+ * host threads (the internal events are shared).
+ */
+size_t attn_fwd_host_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                                    int with_doc_ids);
+attn_status_t attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                            int mask_kind, int window_l, int window_r, int draft_block,
+                            const int32_t* doc_ids, void* workspace, size_t ws_bytes,
+                            void* stream);
+
+/*
  * attn_bwd_workspace_size — bytes of caller workspace attn_bwd needs:
  * an fp32 dQ accumulator [B, Hq, Lq, d] (rounded up to 256 bytes), then fp32
  * D [B, Hq, Lq].  0 for invalid arguments.

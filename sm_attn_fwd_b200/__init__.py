@@ -7,6 +7,7 @@ tensors are not on a CUDA device, the calls raise.
 
 Entry points (same names as the C ABI):
   attn_fwd(q, k, v, ...)                 -> (o, lse)
+  attn_fwd_host(q, k, v, ...)            -> (o, lse)   host tensors in and out
   attn_decode_splitkv(q, k, v, kv_lens, ...) -> (o, lse)
   attn_decode_num_splits(...), attn_decode_workspace_size(...)
   attn_get_device_error(stream=None)     -> (status, raw_bits)
@@ -26,6 +27,7 @@ __all__ = [
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
     "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_bwd", "attn_decode_splitkv",
+    "attn_fwd_host", "attn_fwd_host_workspace_size",
     "attn_decode_num_splits", "SCORE_MOD_NONE", "SCORE_MOD_ALIBI", "SCORE_MOD_REL_BIAS",
     "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
@@ -49,6 +51,7 @@ _MASKS = {"none": MASK_NONE, "causal": MASK_CAUSAL, "draft": MASK_DRAFT_BLOCK}
 
 EXPORTED_SYMBOLS = (
     "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_fwd_varlen_score_mod",
+    "attn_fwd_host_workspace_size", "attn_fwd_host",
     "attn_bwd_workspace_size", "attn_bwd",
     "attn_decode_num_splits", "attn_decode_workspace_size",
     "attn_decode_splitkv", "attn_decode_paged", "attn_decode_splitkv_noalloc",
@@ -88,6 +91,11 @@ def load_library():
         lib.attn_fwd_score_mod.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
                                            i32, i32, i32, P, i32, P, i32, P]
         lib.attn_fwd_score_mod.restype = i32
+        lib.attn_fwd_host_workspace_size.argtypes = [i32] * 7
+        lib.attn_fwd_host_workspace_size.restype = sz
+        lib.attn_fwd_host.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32,
+                                      i32, i32, P, P, sz, P]
+        lib.attn_fwd_host.restype = i32
         lib.attn_bwd_workspace_size.argtypes = [i32, i32, i32, i32]
         lib.attn_bwd_workspace_size.restype = sz
         lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32,
@@ -172,6 +180,57 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
                                  int(draft_block), _ptr(doc_ids), _stream_handle(stream, q.device))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+    return o, lse
+
+
+def _check_host_bf16(name, t):
+    if not isinstance(t, torch.Tensor) or t.device.type != "cpu":
+        raise ValueError(f"{name} must be a host (CPU) tensor")
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous bfloat16 [B, H, L, D] host tensor")
+
+
+def attn_fwd_host_workspace_size(B, Hq, Hkv, Lq, Lk, d, with_doc_ids=False) -> int:
+    return int(load_library().attn_fwd_host_workspace_size(B, Hq, Hkv, Lq, Lk, d,
+                                                           int(bool(with_doc_ids))))
+
+
+def attn_fwd_host(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
+                  doc_ids=None, o=None, lse=None, workspace=None, stream=None, device=None):
+    """attn_fwd on host tensors (see ``attn_fwd_host`` in include/attn.h).
+
+    q, k, v (and doc_ids) are contiguous CPU tensors, pinned for the copies to
+    overlap the kernels; o and lse are CPU tensors (pinned ones are allocated
+    when not given).  The copies and kernels are queued on ``stream``: the
+    outputs are complete once it is synchronised (this wrapper does not wait).
+    Returns (o, lse).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _check_host_bf16(name, t)
+    B, Hq, Lq, d = q.shape
+    _, Hkv, Lk, _ = k.shape
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32).pin_memory()
+    if o.device.type != "cpu" or lse.device.type != "cpu":
+        raise ValueError("o and lse must be host (CPU) tensors")
+    if doc_ids is not None and (doc_ids.dtype != torch.int32 or doc_ids.device.type != "cpu"
+                                or not doc_ids.is_contiguous()):
+        raise ValueError("doc_ids must be a contiguous int32 host tensor [B, Lk]")
+    need = attn_fwd_host_workspace_size(B, Hq, Hkv, Lq, Lk, d, doc_ids is not None)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    mk = mask if isinstance(mask, int) else _MASKS[mask]
+    st = load_library().attn_fwd_host(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Lq, Lk, d, float(scale), mk,
+        int(window[0]), int(window[1]), int(draft_block), _ptr(doc_ids), _ptr(workspace),
+        workspace.numel(), _stream_handle(stream, dev))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_host")
     return o, lse
 
 

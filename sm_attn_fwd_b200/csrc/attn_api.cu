@@ -88,54 +88,103 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Encoded tensor maps are a pure function of their arguments; a small
+// per-thread cache skips the encode (a driver call) when a caller repeats a
+// call on the same buffers and shapes, as decode and training loops do.
+struct TmapKey {
+  const void* base;
+  uint64_t dims[3];
+  int rank, box_rows, kind;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && rank == o.rank && box_rows == o.box_rows && kind == o.kind &&
+           dims[0] == o.dims[0] && dims[1] == o.dims[1] && dims[2] == o.dims[2];
+  }
+};
+constexpr int kTmapCacheSize = 16;
+struct TmapCache {
+  TmapKey key[kTmapCacheSize];
+  CUtensorMap map[kTmapCacheSize];
+  bool valid[kTmapCacheSize] = {};
+  int next = 0;
+};
+thread_local TmapCache t_tmaps;
+
+template <class Encode>
+bool cached_encode(CUtensorMap* map, const TmapKey& key, Encode&& encode) {
+  for (int i = 0; i < kTmapCacheSize; ++i) {
+    if (t_tmaps.valid[i] && t_tmaps.key[i] == key) {
+      *map = t_tmaps.map[i];
+      return true;
+    }
+  }
+  if (!encode(map)) return false;
+  const int slot = t_tmaps.next;
+  t_tmaps.next = (slot + 1) % kTmapCacheSize;
+  t_tmaps.key[slot] = key;
+  t_tmaps.map[slot] = *map;
+  t_tmaps.valid[slot] = true;
+  return true;
+}
+
 // bf16 tensor map of rank 2 or 3 (innermost first), boxes of 64 columns by
 // box_rows rows, 128-byte swizzle; out-of-range rows read as zero.
 bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                  int box_rows = kBlockN) {
-  auto fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t gdim[3];
-  cuuint64_t gstride[2];
-  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
-  cuuint32_t estride[3] = {1, 1, 1};
-  uint64_t stride = 2;
-  for (int i = 0; i < rank; ++i) {
-    gdim[i] = dims[i];
-    if (i > 0) gstride[i - 1] = stride;
-    stride *= dims[i];
-  }
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base),
-                  gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  TmapKey key{base, {dims[0], rank > 1 ? dims[1] : 0, rank > 2 ? dims[2] : 0}, rank, box_rows, 0};
+  return cached_encode(map, key, [&](CUtensorMap* out) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3];
+    cuuint64_t gstride[2];
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t estride[3] = {1, 1, 1};
+    uint64_t stride = 2;
+    for (int i = 0; i < rank; ++i) {
+      gdim[i] = dims[i];
+      if (i > 0) gstride[i - 1] = stride;
+      stride *= dims[i];
+    }
+    CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank,
+                    const_cast<void*>(base), gdim, gstride, box, estride,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+  });
 }
 
 // Token-major packed tensor [total, H, d]: dims {d, H, total}, one head per
 // box row group: box {64 columns, 1 head, 128 tokens}, the same shared-memory
 // image as a 128-row box of the [B, H, L, d] layout.
 bool encode_bf16_packed(CUtensorMap* map, const void* base, int d, int H, int total) {
-  auto fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t gdim[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
-  cuuint64_t gstride[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kBlockN};
-  cuuint32_t estride[3] = {1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3u, const_cast<void*>(base), gdim,
-                  gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  TmapKey key{base, {(uint64_t)d, (uint64_t)H, (uint64_t)total}, 3, kBlockN, 1};
+  return cached_encode(map, key, [&](CUtensorMap* out) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)total};
+    cuuint64_t gstride[2] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kBlockN};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3u, const_cast<void*>(base), gdim,
+                    gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+  });
 }
 
+// SM count of the current device (148 when no device answers), queried once
+// per device and thread.
 int num_sms() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) {
+  thread_local int cached[attn::kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= attn::kMaxDevices) return 148;
+  if (cached[dev] == 0) {
     int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      n = v;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return 148;
+    cached[dev] = v;
   }
-  return n;
+  return cached[dev];
 }
 
 long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
@@ -252,6 +301,13 @@ bool plan_short(int B, int Hq, int Hkv, int Lq, int Lk, int mask_kind, int wl, i
   return true;
 }
 
+bool plan_short_possible(int B, int Hq, int Hkv, int Lq, int Lk, int mask_kind, int wl, int wr,
+                         int draft_block) {
+  ShortPlan sp;
+  return plan_short(B, Hq, Hkv, Lq, Lk, mask_kind, wl, wr,
+                    mask_kind == ATTN_MASK_DRAFT_BLOCK ? draft_block : 1, &sp);
+}
+
 }  // namespace
 
 extern "C" {
@@ -293,10 +349,10 @@ static attn_status_t parse_score_mod(int kind, const float* params, int arg, Sco
   return ATTN_ERR_INVALID_ARG;
 }
 
-static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse,
-                               int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
-                               int mask_kind, int window_l, int window_r, int draft_block,
-                               const int32_t* doc_ids, const ScoreMod& sm, void* stream) {
+static attn_status_t validate_dense(const void* q, const void* k, const void* v, const void* o,
+                                    const float* lse, int B, int Hq, int Hkv, int Lq, int Lk,
+                                    int d, float scale, int mask_kind, int window_l, int window_r,
+                                    int draft_block, const int32_t* doc_ids) {
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       !aligned(lse, 4))
@@ -310,6 +366,21 @@ static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (ceil_div(Lk, kBlockN) > attn::kMaxKvTiles) return ATTN_ERR_UNSUPPORTED;
   if ((long long)B * Hq > kMaxGridY) return ATTN_ERR_UNSUPPORTED;
+  const long long q_tiles = ceil_div(Lq, kBlockM);
+  if ((long long)B * Hq * ((q_tiles + 1) / 2) > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+// allow_short = false keeps every shape on the persistent kernel (the chunks
+// of attn_fwd_host then compute exactly what one attn_fwd call would).
+static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                               int mask_kind, int window_l, int window_r, int draft_block,
+                               const int32_t* doc_ids, const ScoreMod& sm, void* stream,
+                               bool allow_short = true) {
+  const attn_status_t vs = validate_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale,
+                                          mask_kind, window_l, window_r, draft_block, doc_ids);
+  if (vs != ATTN_OK) return vs;
 
   FwdParams p;
   std::memset(&p, 0, sizeof p);
@@ -332,7 +403,6 @@ static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void
   p.scale_log2 = (float)((double)scale * 1.4426950408889634074);
   p.q_tiles = (int)ceil_div(Lq, kBlockM);
   const long long n_units = (long long)B * Hq * ((p.q_tiles + 1) / 2);
-  if (n_units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   p.n_units = (int)n_units;
   p.err = error_word_for_current_device();
   if (!p.err) return ATTN_ERR_CUDA;
@@ -345,7 +415,7 @@ static attn_status_t fwd_dense(const void* q, const void* k, const void* v, void
   // Short queries: a query tile per (b, kv head) leaves most SMs idle in the
   // persistent kernel, so a cluster per row tile splits the visible keys.
   ShortPlan sp;
-  if (!sm.alibi_slopes && !sm.rel_table &&
+  if (allow_short && !sm.alibi_slopes && !sm.rel_table &&
       plan_short(B, Hq, Hkv, Lq, Lk, mask_kind, window_l, window_r, p.draft_block, &sp)) {
     p.row_tiles = sp.row_tiles;
     p.key_lo = sp.key_lo;
@@ -384,6 +454,166 @@ attn_status_t attn_fwd_score_mod(const void* q, const void* k, const void* v, vo
   if (st != ATTN_OK) return st;
   return fwd_dense(q, k, v, o, lse, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
                    draft_block, doc_ids, sm, stream);
+}
+
+// ------------------------------------------------- host buffers, pipelined
+// attn_fwd_host: the inputs and outputs live in host memory.  The work is cut
+// into chunks of whole (b, kv head) pairs (with their query heads); chunk c's
+// Q, K and V go up on one copy stream while the kernel of chunk c - 1 runs on
+// the caller's stream and the O / LSE of chunk c - 2 come down on another, so
+// the PCIe transfers in both directions and the kernels overlap.
+namespace {
+
+constexpr int kHostChunks = 8;  // target chunk count (fewer when B * Hkv is smaller)
+
+struct HostPipe {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t in[kHostChunks] = {}, out[kHostChunks] = {};
+};
+HostPipe g_pipe[attn::kMaxDevices];
+attn::PerContextOnce g_pipe_once;
+std::mutex g_pipe_enqueue;  // the events are reused: one enqueue at a time
+
+struct HostLayout {
+  size_t q, k, v, o, lse, doc, total;
+};
+
+HostLayout host_layout(int B, int Hq, int Hkv, int Lq, int Lk, int d, bool with_doc) {
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  HostLayout l;
+  const size_t qb = (size_t)B * Hq * Lq * d * 2, kb = (size_t)B * Hkv * Lk * d * 2;
+  l.q = 0;
+  l.k = up(qb);
+  l.v = l.k + up(kb);
+  l.o = l.v + up(kb);
+  l.lse = l.o + up(qb);
+  l.doc = l.lse + up((size_t)B * Hq * Lq * 4);
+  l.total = l.doc + (with_doc ? up((size_t)B * Lk * 4) : 0);
+  return l;
+}
+
+// A chunk: batch elements [b0, b0 + nb) times kv heads [h0, h0 + nh).
+struct HostChunk {
+  int b0, nb, h0, nh;
+};
+
+int plan_host_chunks(int B, int Hkv, HostChunk* out) {
+  int n = 0;
+  if (B >= kHostChunks) {
+    const int nb = (B + kHostChunks - 1) / kHostChunks;
+    for (int b0 = 0; b0 < B; b0 += nb) out[n++] = {b0, std::min(nb, B - b0), 0, Hkv};
+  } else {
+    const int parts = std::min(Hkv, kHostChunks / B);
+    const int nh = (Hkv + parts - 1) / parts;
+    for (int b = 0; b < B; ++b)
+      for (int h0 = 0; h0 < Hkv; h0 += nh) out[n++] = {b, 1, h0, std::min(nh, Hkv - h0)};
+  }
+  return n;
+}
+
+}  // namespace
+
+size_t attn_fwd_host_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int d,
+                                    int with_doc_ids) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || d < 1 || Hq % Hkv != 0) return 0;
+  return host_layout(B, Hq, Hkv, Lq, Lk, d, with_doc_ids != 0).total;
+}
+
+attn_status_t attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Lq, int Lk, int d, float scale,
+                            int mask_kind, int window_l, int window_r, int draft_block,
+                            const int32_t* doc_ids, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Lq < 1 || Lk < 1 || d < 1 || Hq % Hkv != 0)
+    return ATTN_ERR_INVALID_ARG;
+  const HostLayout lay = host_layout(B, Hq, Hkv, Lq, Lk, d, doc_ids != nullptr);
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < lay.total) return ATTN_ERR_WORKSPACE;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  uint8_t *qd = ws + lay.q, *kd = ws + lay.k, *vd = ws + lay.v, *od = ws + lay.o;
+  float* ld = reinterpret_cast<float*>(ws + lay.lse);
+  int32_t* dd = doc_ids ? reinterpret_cast<int32_t*>(ws + lay.doc) : nullptr;
+  // the whole call's arguments, checked on the device-side copies before any work is queued
+  const attn_status_t vs = validate_dense(qd, kd, vd, od, ld, B, Hq, Hkv, Lq, Lk, d, scale,
+                                          mask_kind, window_l, window_r, draft_block, dd);
+  if (vs != ATTN_OK) return vs;
+  // chunks stay on the kernel one call over the whole shape would use, so the
+  // results match attn_fwd exactly; short-query shapes run as one chunk
+  const bool whole_short =
+      plan_short_possible(B, Hq, Hkv, Lq, Lk, mask_kind, window_l, window_r, draft_block);
+  HostChunk chunks[kHostChunks * 2];
+  const int n_chunks = whole_short ? 1 : plan_host_chunks(B, Hkv, chunks);
+  if (whole_short) chunks[0] = {0, B, 0, Hkv};
+
+  const cudaError_t se = attn::once_per_context(g_pipe_once, [](int dev) {
+    HostPipe& hp = g_pipe[dev];
+    cudaError_t e = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.done, cudaEventDisableTiming);
+    for (int i = 0; i < kHostChunks && e == cudaSuccess; ++i) {
+      e = cudaEventCreateWithFlags(&hp.in[i], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hp.out[i], cudaEventDisableTiming);
+    }
+    return e;
+  });
+  if (se != cudaSuccess) return ATTN_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  HostPipe& hp = g_pipe[dev];
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int group = Hq / Hkv;
+  const size_t qrow = (size_t)Lq * d * 2, krow = (size_t)Lk * d * 2;  // bytes per head
+
+  std::lock_guard<std::mutex> lock(g_pipe_enqueue);
+  bool ok = cudaEventRecord(hp.start, st) == cudaSuccess &&
+            cudaStreamWaitEvent(hp.h2d, hp.start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(hp.d2h, hp.start, 0) == cudaSuccess;
+  if (ok && doc_ids)
+    ok = cudaMemcpyAsync(dd, doc_ids, (size_t)B * Lk * 4, cudaMemcpyHostToDevice, hp.h2d) ==
+         cudaSuccess;
+  for (int c = 0; c < n_chunks && ok; ++c) {
+    const HostChunk& ch = chunks[c];
+    const size_t qh0 = (size_t)ch.b0 * Hq + (size_t)ch.h0 * group;   // first query head
+    const size_t kh0 = (size_t)ch.b0 * Hkv + (size_t)ch.h0;          // first kv head
+    const size_t nq = (size_t)ch.nb * ch.nh * group, nk = (size_t)ch.nb * ch.nh;
+    ok = cudaMemcpyAsync(qd + qh0 * qrow, static_cast<const uint8_t*>(q) + qh0 * qrow, nq * qrow,
+                         cudaMemcpyHostToDevice, hp.h2d) == cudaSuccess &&
+         cudaMemcpyAsync(kd + kh0 * krow, static_cast<const uint8_t*>(k) + kh0 * krow, nk * krow,
+                         cudaMemcpyHostToDevice, hp.h2d) == cudaSuccess &&
+         cudaMemcpyAsync(vd + kh0 * krow, static_cast<const uint8_t*>(v) + kh0 * krow, nk * krow,
+                         cudaMemcpyHostToDevice, hp.h2d) == cudaSuccess &&
+         cudaEventRecord(hp.in[c], hp.h2d) == cudaSuccess;
+  }
+  attn_status_t status = ok ? ATTN_OK : ATTN_ERR_CUDA;
+  for (int c = 0; c < n_chunks && status == ATTN_OK; ++c) {
+    const HostChunk& ch = chunks[c];
+    const size_t qh0 = (size_t)ch.b0 * Hq + (size_t)ch.h0 * group;
+    const size_t kh0 = (size_t)ch.b0 * Hkv + (size_t)ch.h0;
+    const size_t nq = (size_t)ch.nb * ch.nh * group;
+    if (cudaStreamWaitEvent(st, hp.in[c], 0) != cudaSuccess) {
+      status = ATTN_ERR_CUDA;
+      break;
+    }
+    status = fwd_dense(qd + qh0 * qrow, kd + kh0 * krow, vd + kh0 * krow, od + qh0 * qrow,
+                       ld + qh0 * Lq, ch.nb, ch.nh * group, ch.nh, Lq, Lk, d, scale, mask_kind,
+                       window_l, window_r, draft_block, dd ? dd + (size_t)ch.b0 * Lk : nullptr,
+                       ScoreMod{}, stream, whole_short);
+    if (status != ATTN_OK) break;
+    if (cudaEventRecord(hp.out[c], st) != cudaSuccess ||
+        cudaStreamWaitEvent(hp.d2h, hp.out[c], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(o) + qh0 * qrow, od + qh0 * qrow, nq * qrow,
+                        cudaMemcpyDeviceToHost, hp.d2h) != cudaSuccess ||
+        cudaMemcpyAsync(lse + qh0 * Lq, ld + qh0 * Lq, nq * Lq * 4, cudaMemcpyDeviceToHost,
+                        hp.d2h) != cudaSuccess)
+      status = ATTN_ERR_CUDA;
+  }
+  // the caller's stream resumes after the last download, whatever happened above
+  if (cudaEventRecord(hp.done, hp.d2h) != cudaSuccess ||
+      cudaStreamWaitEvent(st, hp.done, 0) != cudaSuccess)
+    status = ATTN_ERR_CUDA;
+  return status;
 }
 
 static attn_status_t fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,

@@ -185,6 +185,38 @@ def test_attn_bwd_rejects_on_host_and_sizes_its_workspace():
     assert lib.attn_bwd(*ptrs, *bad_ws) == ab.ATTN_ERR_INVALID_ARG
 
 
+def test_attn_fwd_host_sizes_its_workspace_and_rejects_on_host():
+    lib = ab.load_library()
+    B, Hq, Hkv, Lq, Lk, d = 2, 8, 2, 100, 130, 64
+
+    def up(x):
+        return (x + 255) // 256 * 256
+    qb, kb = B * Hq * Lq * d * 2, B * Hkv * Lk * d * 2
+    base = up(qb) + 2 * up(kb) + up(qb) + up(B * Hq * Lq * 4)
+    assert lib.attn_fwd_host_workspace_size(B, Hq, Hkv, Lq, Lk, d, 0) == base
+    assert lib.attn_fwd_host_workspace_size(B, Hq, Hkv, Lq, Lk, d, 1) == base + up(B * Lk * 4)
+    assert lib.attn_fwd_host_workspace_size(B, 7, Hkv, Lq, Lk, d, 0) == 0
+    h = ctypes.c_void_p(0x1000)   # host pointers are only passed to copies; nothing is queued
+    args = [h, h, h, h, h, B, Hq, Hkv, Lq, Lk, d, 0.125, 1, -1, -1, 1, None]
+    assert lib.attn_fwd_host(*args, None, 0, None) == ab.ATTN_ERR_WORKSPACE
+    assert lib.attn_fwd_host(*args, ctypes.c_void_p(0x10010), base, None) == ab.ATTN_ERR_WORKSPACE
+    assert lib.attn_fwd_host(*args, A, base - 1, None) == ab.ATTN_ERR_WORKSPACE
+    bad = list(args)
+    bad[6] = 3                                                            # Hq % Hkv != 0
+    assert lib.attn_fwd_host(*bad, A, base, None) == ab.ATTN_ERR_INVALID_ARG
+    bad = list(args)
+    bad[10] = 96                                                          # d
+    assert lib.attn_fwd_host(*bad, A, 1 << 30, None) == ab.ATTN_ERR_UNSUPPORTED
+    bad = list(args)
+    bad[12] = 7                                                           # mask kind
+    assert lib.attn_fwd_host(*bad, A, base, None) == ab.ATTN_ERR_INVALID_ARG
+    with pytest.raises(ValueError, match="host"):
+        import torch
+        ab.attn_fwd_host(torch.zeros(1, 2, 8, 64, dtype=torch.float32),
+                         torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16),
+                         torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16))
+
+
 def test_binding_checks_tensors_before_calling_the_library():
     """The Python binding rejects host tensors, wrong dtypes and wrong ranks itself."""
     import torch

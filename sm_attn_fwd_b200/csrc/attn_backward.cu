@@ -60,8 +60,10 @@ struct BwdCfg {
   static constexpr int kOffQ = kOffV + kTileBytes;          // [kQBufs]
   static constexpr int kOffDO = kOffQ + kQBufs * kTileBytes;  // [kQBufs]
   static constexpr int kOffDS = kOffDO + kQBufs * kTileBytes;  // dS^T: [128 keys][128 queries] bf16
-  static constexpr int kOffStat = kOffDS + 2 * kAtomBytes;     // [kQBufs] x (lse2, dsum, qdoc)
-  static constexpr int kOffBar = kOffStat + kQBufs * 3 * 128 * 4;
+  // per buffer: -LSE2 [128], -D [128], qdoc [128], the tile's qdoc min and max, padding
+  static constexpr int kStatWords = 400;
+  static constexpr int kOffStat = kOffDS + 2 * kAtomBytes;     // [kQBufs] x kStatWords
+  static constexpr int kOffBar = kOffStat + kQBufs * kStatWords * 4;
   static constexpr int kNumBars = 12;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
@@ -137,10 +139,16 @@ __global__ void attn_bwd_dsum_kernel(const BwdParams p) {
   if (lane == 0) p.dsum[row] = acc;
 }
 
-// dQ (bf16) from its fp32 accumulator.
-__global__ void attn_bwd_dq_kernel(const BwdParams p, long long n) {
+// dQ (bf16) from its fp32 accumulator, four elements per thread (n4 = n / 4;
+// n is a multiple of 64).
+__global__ void attn_bwd_dq_kernel(const BwdParams p, long long n4) {
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) reinterpret_cast<__nv_bfloat16*>(p.dq)[i] = __float2bfloat16_rn(p.dq_acc[i]);
+  if (i >= n4) return;
+  const float4 v = reinterpret_cast<const float4*>(p.dq_acc)[i];
+  uint2 out;
+  out.x = ptx::pack_bf16x2(v.x, v.y);
+  out.y = ptx::pack_bf16x2(v.z, v.w);
+  reinterpret_cast<uint2*>(p.dq)[i] = out;
 }
 
 template <int D>
@@ -228,24 +236,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
-      // row statistics of the query tile: LSE in base 2 (+inf for rows past Lq
-      // or with no visible key, so their P is 0), D, and the rows' documents
-      float* lse2_s = stat_s + slot * 384;
-      float* dsum_s = lse2_s + 128;
-      int* qdoc_s = reinterpret_cast<int*>(dsum_s + 128);
+      // row statistics of the query tile, negated for the packed FMA and add of
+      // the softmax warps: -LSE in base 2 (-inf for rows past Lq or with no
+      // visible key, so their P is exactly 0), -D; the rows' documents and
+      // their min / max over the tile
+      float* nl2_s = stat_s + slot * C::kStatWords;
+      float* nds_s = nl2_s + 128;
+      int* qdoc_s = reinterpret_cast<int*>(nds_s + 128);
+      int dmin = 0x7fffffff, dmax = (int)0x80000000;
       for (int r = lane; r < 128; r += 32) {
         const int qi = q0 + r;
-        float l2 = INFINITY, dd = 0.0f;
+        float nl2 = -INFINITY, nds = 0.0f;
         int qd = 0;
         if (qi < p.Lq) {
           const float lse = __ldg(p.lse + bh * p.Lq + qi);
-          l2 = (lse == -INFINITY) ? INFINITY : lse * kLog2eB;
-          dd = __ldg(p.dsum + bh * p.Lq + qi);
-          if (p.doc_ids != nullptr) qd = __ldg(p.doc_ids + (long long)b * p.Lk + (p.Lk - p.Lq + qi));
+          nl2 = (lse == -INFINITY) ? -INFINITY : -(lse * kLog2eB);
+          nds = -__ldg(p.dsum + bh * p.Lq + qi);
+          if (p.doc_ids != nullptr) {
+            qd = __ldg(p.doc_ids + (long long)b * p.Lk + (p.Lk - p.Lq + qi));
+            dmin = min(dmin, qd);
+            dmax = max(dmax, qd);
+          }
         }
-        lse2_s[r] = l2;
-        dsum_s[r] = dd;
+        nl2_s[r] = nl2;
+        nds_s[r] = nds;
         qdoc_s[r] = qd;
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        dmin = min(dmin, __shfl_xor_sync(0xffffffffu, dmin, o));
+        dmax = max(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+      }
+      if (lane == 0) {
+        qdoc_s[128] = dmin;
+        qdoc_s[129] = dmax;
       }
       __syncwarp();
       if (lane == 0) {
@@ -337,37 +360,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int q0 = iter_q0(it);
       if (!pair_live(p, k0, q0)) continue;
       const int hq = iter_hq(it);
-      const float* lse2_s = stat_s + (n % QB) * 384;
-      const float* dsum_s = lse2_s + 128;
-      const int* qdoc_s = reinterpret_cast<const int*>(dsum_s + 128);
+      const uint32_t stats = ptx::smem_u32(stat_s + (n % QB) * C::kStatWords);
+      const int* qdoc_s = reinterpret_cast<const int*>(stat_s + (n % QB) * C::kStatWords + 256);
       ok = ptx::mbar_wait_a(BAR(kBarSFull), (uint32_t)n & 1u, abort_flag, err,
                             kDevErrTimeoutSoftmax);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
+      // every key of the warp sees every query row of the tile: no mask code
+      // (rows past Lq carry -LSE2 = -inf, so their P is 0 either way)
+      bool sees_all = key < p.Lk && qlo <= q0 && qhi >= q0 + 127;
+      if (p.doc_ids != nullptr) sees_all = sees_all && qdoc_s[128] == kdoc && qdoc_s[129] == kdoc;
+      const bool full = __all_sync(0xffffffffu, sees_all);
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {  // 32 query columns at a time
         uint32_t rs[32], rd[32];
         ptx::tmem_ld32(t_row + C::kST + cc * 32, rs);
         ptx::tmem_ld32(t_row + C::kDPT + cc * 32, rd);
+        float nl[32], nd[32];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint32_t w0, w1, w2, w3;
+          ptx::ld_shared_v4(stats + (uint32_t)(cc * 128 + j * 16), w0, w1, w2, w3);
+          nl[4 * j] = __uint_as_float(w0);
+          nl[4 * j + 1] = __uint_as_float(w1);
+          nl[4 * j + 2] = __uint_as_float(w2);
+          nl[4 * j + 3] = __uint_as_float(w3);
+          ptx::ld_shared_v4(stats + (uint32_t)(512 + cc * 128 + j * 16), w0, w1, w2, w3);
+          nd[4 * j] = __uint_as_float(w0);
+          nd[4 * j + 1] = __uint_as_float(w1);
+          nd[4 * j + 2] = __uint_as_float(w2);
+          nd[4 * j + 3] = __uint_as_float(w3);
+        }
+        if (!full) {
+          // masked: an invisible pair gets -LSE2 = -inf, so its P (and dS) is 0
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int qi = q0 + cc * 32 + i;
+            bool vis = qi >= qlo && qi <= qhi;
+            if (p.doc_ids != nullptr) vis = vis && (qdoc_s[cc * 32 + i] == kdoc);
+            nl[i] = vis ? nl[i] : -INFINITY;
+          }
+        }
         ptx::tmem_wait_ld();
         uint32_t pp[16], dp[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2) {
-          float pv[2], dv[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int col = cc * 32 + i + h;
-            const int qi = q0 + col;
-            bool vis = qi >= qlo && qi <= qhi;
-            if (p.doc_ids != nullptr) vis = vis && (qdoc_s[col] == kdoc);
-            const float l2 = lse2_s[col];
-            const float pe = vis ? ptx::ex2(__uint_as_float(rs[i + h]) * c - l2) : 0.0f;
-            pv[h] = (l2 == INFINITY) ? 0.0f : pe;
-            dv[h] = pv[h] * (__uint_as_float(rd[i + h]) - dsum_s[col]);
-          }
-          pp[i / 2] = ptx::pack_bf16x2(pv[0], pv[1]);
-          dp[i / 2] = ptx::pack_bf16x2(dv[0], dv[1]);
+          // P = 2^(S c - LSE2), dS = P (dP - D), two query columns per packed op
+          float x0, x1, d0, d1;
+          ptx::fma2_bv(x0, x1, __uint_as_float(rs[i]), __uint_as_float(rs[i + 1]), c, nl[i],
+                       nl[i + 1]);
+          const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+          ptx::addmul2(d0, d1, __uint_as_float(rd[i]), __uint_as_float(rd[i + 1]), nd[i],
+                       nd[i + 1], p0, p1);
+          pp[i / 2] = ptx::pack_bf16x2(p0, p1);
+          dp[i / 2] = ptx::pack_bf16x2(d0, d1);
         }
         // P^T and dS^T over the columns already read (16 columns per 32 queries)
         ptx::tmem_st16(t_row + C::kST + cc * 16, pp);
@@ -484,8 +531,8 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const long long n = nrows * D;
-  attn_bwd_dq_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p, n);
+  const long long n4 = nrows * D / 4;
+  attn_bwd_dq_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(p, n4);
   return cudaGetLastError();
 }
 

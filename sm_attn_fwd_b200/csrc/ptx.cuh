@@ -463,6 +463,29 @@ __device__ __forceinline__ void add2_acc(float& s0, float& s1, float a0, float a
       : "f"(a0), "f"(a1));
 }
 
+// (d0, d1) = (a0 + b0, a1 + b1) * (m0, m1): one packed add, one packed multiply
+// (each rounded to nearest, as the scalar pair would be).
+__device__ __forceinline__ void addmul2(float& d0, float& d1, float a0, float a1, float b0,
+                                        float b1, float m0, float m1) {
+  asm("{\n\t.reg .b64 ra, rb, rm, rt;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rm, {%6, %7};\n\t"
+      "add.rn.f32x2 rt, ra, rb;\n\t"
+      "mul.rn.f32x2 rt, rt, rm;\n\t"
+      "mov.b64 {%0, %1}, rt;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(m0), "f"(m1));
+}
+
+// Four consecutive 32-bit words from shared memory (16-byte aligned address).
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
+                                             uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a), "=r"(b), "=r"(c), "=r"(d)
+               : "r"(addr));
+}
+
 // Maximum of 128 values: sixteen independent chains of two-input max, then a tree.
 __device__ __forceinline__ float row_max128(const float (&v)[128]) {
   float m[16];

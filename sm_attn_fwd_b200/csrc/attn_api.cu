@@ -29,7 +29,8 @@ cudaError_t launch_prefill(const CUtensorMap&, const CUtensorMap&, const CUtenso
 int* device_error_word();
 template <int D>
 cudaError_t launch_backward(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
-                            const CUtensorMap&, const BwdParams&, cudaStream_t);
+                            const CUtensorMap&, const CUtensorMap&, const BwdParams&,
+                            cudaStream_t);
 cudaError_t launch_selftest_wait(cudaStream_t stream);
 template <int D>
 cudaError_t launch_short(const CUtensorMap&, const CUtensorMap&, const CUtensorMap&,
@@ -148,6 +149,25 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
                     const_cast<void*>(base), gdim, gstride, box, estride,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+  });
+}
+
+// fp32 tensor of rank 3 {cols, rows, planes} for bulk reduce-adds from shared
+// memory: boxes of 32 columns (128 bytes) by 128 rows, 128-byte swizzle.
+bool encode_f32_reduce(CUtensorMap* map, const void* base, const uint64_t* dims) {
+  TmapKey key{base, {dims[0], dims[1], dims[2]}, 3, kBlockN, 2};
+  return cached_encode(map, key, [&](CUtensorMap* out) {
+    auto fn = get_encode_fn();
+    if (!fn) return false;
+    cuuint64_t gdim[3] = {dims[0], dims[1], dims[2]};
+    cuuint64_t gstride[2] = {dims[0] * 4, dims[0] * dims[1] * 4};
+    cuuint32_t box[3] = {32, (cuuint32_t)kBlockN, 1};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3u, const_cast<void*>(base), gdim,
+                    gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
   });
 }
@@ -759,16 +779,17 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   p.err = error_word_for_current_device();
   if (!p.err) return ATTN_ERR_CUDA;
 
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   const uint64_t dq3[3] = {(uint64_t)d, (uint64_t)Lq, (uint64_t)B * Hq};
   const uint64_t dk3[3] = {(uint64_t)d, (uint64_t)Lk, (uint64_t)B * Hkv};
   if (!encode_bf16(&tq, q, 3, dq3) || !encode_bf16(&tk, k, 3, dk3) ||
-      !encode_bf16(&tv, v, 3, dk3) || !encode_bf16(&tdo, dout, 3, dq3))
+      !encode_bf16(&tv, v, 3, dk3) || !encode_bf16(&tdo, dout, 3, dq3) ||
+      !encode_f32_reduce(&tdq, p.dq_acc, dq3))
     return ATTN_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(p.dq_acc, 0, rows * (size_t)d * 4, st) != cudaSuccess) return ATTN_ERR_CUDA;
-  cudaError_t e = d == 64 ? attn::launch_backward<64>(tq, tk, tv, tdo, p, st)
-                          : attn::launch_backward<128>(tq, tk, tv, tdo, p, st);
+  cudaError_t e = d == 64 ? attn::launch_backward<64>(tq, tk, tv, tdo, tdq, p, st)
+                          : attn::launch_backward<128>(tq, tk, tv, tdo, tdq, p, st);
   return e == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

@@ -63,7 +63,11 @@ struct BwdCfg {
   // per buffer: -LSE2 [128], -D [128], qdoc [128], the tile's qdoc min and max, padding
   static constexpr int kStatWords = 400;
   static constexpr int kOffStat = kOffDS + 2 * kAtomBytes;     // [kQBufs] x kStatWords
-  static constexpr int kOffBar = kOffStat + kQBufs * kStatWords * 4;
+  // dQ staging: 64 columns of fp32 as two 128-byte-swizzled boxes of 32 columns
+  // by 128 rows, reduced into the accumulator by TMA (d = 128: two rounds)
+  static constexpr int kOffStage = (kOffStat + kQBufs * kStatWords * 4 + 1023) / 1024 * 1024;
+  static constexpr int kStageBoxBytes = 128 * 128;
+  static constexpr int kOffBar = kOffStage + 2 * kStageBoxBytes;
   static constexpr int kNumBars = 12;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16;
@@ -77,7 +81,8 @@ struct BwdCfg {
 };
 
 enum : int { kBarKv = 0, kBarQFull, kBarQFull1, kBarQEmpty, kBarQEmpty1, kBarSFull, kBarPFull,
-             kBarDqFull, kBarDqFree, kBarAcc };
+             kBarDqFull, kBarDqFree, kBarAcc, kBarStageFull, kBarStageFree };
+constexpr int kStageIssuer = 64;  // thread that issues the dQ reduce-adds (warp 2, lane 0)
 
 __device__ __forceinline__ uint64_t bdesc(uint32_t addr, uint32_t lbo_bytes) {
   return ptx::smem_desc_sw128(addr, lbo_bytes, 1024);
@@ -155,7 +160,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using C = BwdCfg<D>;
   constexpr int QB = C::kQBufs;
   extern __shared__ uint8_t smem_raw[];
@@ -166,6 +171,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t sq = ptx::smem_u32(smem + C::kOffQ);
   const uint32_t sdo = ptx::smem_u32(smem + C::kOffDO);
   const uint32_t sds = ptx::smem_u32(smem + C::kOffDS);
+  const uint32_t sstage = ptx::smem_u32(smem + C::kOffStage);
   // row statistics of buffer slot: lse2 [128], dsum [128], qdoc [128]
   float* stat_s = reinterpret_cast<float*>(smem + C::kOffStat);
   const uint32_t bar0 = ptx::smem_u32(smem + C::kOffBar);
@@ -186,6 +192,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ptx::prefetch_tmap(&tm_k);
     ptx::prefetch_tmap(&tm_v);
     ptx::prefetch_tmap(&tm_do);
+    ptx::prefetch_tmap(&tm_dq);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     ptx::mbar_init(&bars[kBarKv], 1);
     for (int i = 0; i < 2; ++i) {
@@ -197,6 +204,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     ptx::mbar_init(&bars[kBarDqFull], 1);
     ptx::mbar_init(&bars[kBarDqFree], 128);
     ptx::mbar_init(&bars[kBarAcc], 1);
+    ptx::mbar_init(&bars[kBarStageFull], 128);
+    ptx::mbar_init(&bars[kBarStageFree], 1);
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -435,36 +444,73 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ptx::fence_proxy_async_smem();
       ptx::tc_fence_before();
       ptx::mbar_arrive_a(BAR(kBarPFull));
-      // dQ tile: TMEM lane = query of the tile; reduce scale * dQ into the accumulator
+      // dQ tile: TMEM lane = query of the tile.  scale * dQ goes through a
+      // 32 KB staging tile in shared memory (64 columns per round: one round
+      // for d = 64, two for d = 128) and is added into the fp32 accumulator by
+      // two TMA bulk reduce-adds per round, issued by one thread; the staging
+      // tile is rewritten only after the previous round's reduce has read it.
       ok = ptx::mbar_wait_a(BAR(kBarDqFull), (uint32_t)n & 1u, abort_flag, err,
                             kDevErrTimeoutSoftmax);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       ptx::tc_fence_after();
-      const int qi = q0 + row;
-      float* dst = p.dq_acc + (((long long)b * p.Hq + hq) * p.Lq + qi) * D;
+      const long long bh = (long long)b * p.Hq + hq;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        // columns of d [32 cc, 32 cc + 32): first and second 64-column half
-        const uint32_t col = (cc < 2 ? C::kDQ0 : C::kDQ1) + (uint32_t)((cc & 1) * 32);
-        uint32_t r[32];
-        ptx::tmem_ld32(t_row + (D == 64 ? C::kDQ0 + (uint32_t)(cc * 32) : col), r);
-        ptx::tmem_wait_ld();
-        if (qi < p.Lq) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + cc * 32 + i),
-                         "f"(__uint_as_float(r[i]) * p.scale),
-                         "f"(__uint_as_float(r[i + 1]) * p.scale),
-                         "f"(__uint_as_float(r[i + 2]) * p.scale),
-                         "f"(__uint_as_float(r[i + 3]) * p.scale)
-                         : "memory");
+      for (int h = 0; h < D / 64 && ok; ++h) {
+        const int g = n * (D / 64) + h;  // staging round
+        if (g > 0) {
+          if (threadIdx.x == kStageIssuer) {
+            ptx::bulk_wait_group_read0();
+            ptx::mbar_arrive_a(BAR(kBarStageFree));
+          }
+          ok = ptx::mbar_wait_a(BAR(kBarStageFree), (uint32_t)(g - 1) & 1u, abort_flag, err,
+                                kDevErrTimeoutSoftmax);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
         }
+#pragma unroll 1
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int cb = h * 2 + c2;  // 32-column block of d
+          // columns of d [32 cb, 32 cb + 32): first and second 64-column half
+          const uint32_t col = D == 64 ? C::kDQ0 + (uint32_t)(cb * 32)
+                                       : (cb < 2 ? C::kDQ0 : C::kDQ1) + (uint32_t)((cb & 1) * 32);
+          uint32_t r[32];
+          ptx::tmem_ld32(t_row + col, r);
+          ptx::tmem_wait_ld();
+          if (cb == D / 32 - 1) {  // the dQ columns are read out
+            ptx::tc_fence_before();
+            ptx::mbar_arrive_a(BAR(kBarDqFree));
+          }
+          const uint32_t rowp = sstage + (uint32_t)(c2 * C::kStageBoxBytes) + (uint32_t)row * 128u;
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t addr = rowp + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4);
+            asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                         "f"(__uint_as_float(r[4 * ch]) * p.scale),
+                         "f"(__uint_as_float(r[4 * ch + 1]) * p.scale),
+                         "f"(__uint_as_float(r[4 * ch + 2]) * p.scale),
+                         "f"(__uint_as_float(r[4 * ch + 3]) * p.scale)
+                         : "memory");
+          }
+        }
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive_a(BAR(kBarStageFull));
+        if (threadIdx.x == kStageIssuer) {
+          ok = ptx::mbar_wait_a(BAR(kBarStageFull), (uint32_t)g & 1u, abort_flag, err,
+                                kDevErrTimeoutSoftmax);
+          if (ok) {
+            // rows past Lq fall outside the map and are not written
+            ptx::tma_reduce_add_3d(&tm_dq, sstage, h * 64, q0, (int)bh);
+            ptx::tma_reduce_add_3d(&tm_dq, sstage + C::kStageBoxBytes, h * 64 + 32, q0, (int)bh);
+            ptx::bulk_commit_group();
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok);
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive_a(BAR(kBarDqFree));
       ++n;
     }
+    // the last reduce-adds are complete before the CTA exits
+    if (threadIdx.x == kStageIssuer) ptx::bulk_wait_group0();
     // dK (times scale) and dV of this key tile
     if (ok) {
       ok = ptx::mbar_wait_a(BAR(kBarAcc), 0, abort_flag, err, kDevErrTimeoutSoftmax);
@@ -515,7 +561,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // caller zeroes dq_acc before (on the same stream).
 template <int D>
 cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+                            const CUtensorMap& tdo, const CUtensorMap& tdq, const BwdParams& p,
+                            cudaStream_t stream) {
   const long long nrows = (long long)p.B * p.Hq * p.Lq;
   attn_bwd_dsum_kernel<D><<<(unsigned)((nrows + 7) / 8), 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
@@ -528,7 +575,7 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   });
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)((p.Lk + 127) / 128), (unsigned)(p.B * p.Hkv), 1);
-  kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long n4 = nrows * D / 4;
@@ -538,9 +585,9 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
 
 template cudaError_t launch_backward<64>(const CUtensorMap&, const CUtensorMap&,
                                          const CUtensorMap&, const CUtensorMap&,
-                                         const BwdParams&, cudaStream_t);
+                                         const CUtensorMap&, const BwdParams&, cudaStream_t);
 template cudaError_t launch_backward<128>(const CUtensorMap&, const CUtensorMap&,
                                           const CUtensorMap&, const CUtensorMap&,
-                                          const BwdParams&, cudaStream_t);
+                                          const CUtensorMap&, const BwdParams&, cudaStream_t);
 
 }  // namespace attn

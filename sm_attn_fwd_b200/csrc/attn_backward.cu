@@ -232,10 +232,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ptx::tma_load_3d_a(sv + a * C::kAtomBytes, &tm_v, BAR(kBarKv), a * 64, k0, b * p.Hkv + hkv);
       }
     }
-    int n = 0;  // live pairs so far
-    for (int it = 0; it < n_iter && ok; ++it) {
+    // The row statistics of the next live query tile (this lane's rows r =
+    // lane + 32 m) are loaded into registers while the producer waits for its
+    // buffer, so the Q / dO loads go out as soon as the buffer is free.
+    auto next_live = [&](int it) {
+      while (it < n_iter && !pair_live(p, k0, iter_q0(it))) ++it;
+      return it;
+    };
+    float f_nl2[4], f_nds[4];
+    int f_doc[4];
+    auto fetch = [&](int it) {
       const int q0 = iter_q0(it);
-      if (!pair_live(p, k0, q0)) continue;
+      const long long bh = (long long)b * p.Hq + iter_hq(it);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int qi = q0 + lane + 32 * m;
+        f_nl2[m] = -INFINITY;
+        f_nds[m] = 0.0f;
+        f_doc[m] = 0;
+        if (it < n_iter && qi < p.Lq) {
+          const float lse = __ldg(p.lse + bh * p.Lq + qi);
+          f_nl2[m] = (lse == -INFINITY) ? -INFINITY : -(lse * kLog2eB);
+          f_nds[m] = -__ldg(p.dsum + bh * p.Lq + qi);
+          if (p.doc_ids != nullptr)
+            f_doc[m] = __ldg(p.doc_ids + (long long)b * p.Lk + (p.Lk - p.Lq + qi));
+        }
+      }
+    };
+    int n = 0;  // live pairs so far
+    int it = next_live(0);
+    fetch(it);
+    while (it < n_iter && ok) {
+      const int q0 = iter_q0(it);
       const int hq = iter_hq(it);
       const long long bh = (long long)b * p.Hq + hq;
       const int slot = n % QB;
@@ -245,6 +273,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
       }
+      if (lane == 0) {
+        ptx::mbar_expect_tx_a(BAR(kBarQFull + slot), 2 * kTx);
+        for (int a = 0; a < D / 64; ++a) {
+          ptx::tma_load_3d_a(sq + slot * C::kTileBytes + a * C::kAtomBytes, &tm_q,
+                             BAR(kBarQFull + slot), a * 64, q0, (int)bh);
+          ptx::tma_load_3d_a(sdo + slot * C::kTileBytes + a * C::kAtomBytes, &tm_do,
+                             BAR(kBarQFull + slot), a * 64, q0, (int)bh);
+        }
+      }
       // row statistics of the query tile, negated for the packed FMA and add of
       // the softmax warps: -LSE in base 2 (-inf for rows past Lq or with no
       // visible key, so their P is exactly 0), -D; the rows' documents and
@@ -253,43 +290,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       float* nds_s = nl2_s + 128;
       int* qdoc_s = reinterpret_cast<int*>(nds_s + 128);
       int dmin = 0x7fffffff, dmax = (int)0x80000000;
-      for (int r = lane; r < 128; r += 32) {
-        const int qi = q0 + r;
-        float nl2 = -INFINITY, nds = 0.0f;
-        int qd = 0;
-        if (qi < p.Lq) {
-          const float lse = __ldg(p.lse + bh * p.Lq + qi);
-          nl2 = (lse == -INFINITY) ? -INFINITY : -(lse * kLog2eB);
-          nds = -__ldg(p.dsum + bh * p.Lq + qi);
-          if (p.doc_ids != nullptr) {
-            qd = __ldg(p.doc_ids + (long long)b * p.Lk + (p.Lk - p.Lq + qi));
-            dmin = min(dmin, qd);
-            dmax = max(dmax, qd);
-          }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = lane + 32 * m;
+        nl2_s[r] = f_nl2[m];
+        nds_s[r] = f_nds[m];
+        qdoc_s[r] = f_doc[m];
+        if (q0 + r < p.Lq) {
+          dmin = min(dmin, f_doc[m]);
+          dmax = max(dmax, f_doc[m]);
         }
-        nl2_s[r] = nl2;
-        nds_s[r] = nds;
-        qdoc_s[r] = qd;
       }
       for (int o = 16; o > 0; o >>= 1) {
         dmin = min(dmin, __shfl_xor_sync(0xffffffffu, dmin, o));
         dmax = max(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
       }
       if (lane == 0) {
-        qdoc_s[128] = dmin;
-        qdoc_s[129] = dmax;
+        qdoc_s[128] = p.doc_ids != nullptr ? dmin : 0;
+        qdoc_s[129] = p.doc_ids != nullptr ? dmax : 0;
       }
       __syncwarp();
-      if (lane == 0) {
-        ptx::mbar_arrive_expect_tx_a(BAR(kBarQFull + slot), 2 * kTx);
-        for (int a = 0; a < D / 64; ++a) {
-          ptx::tma_load_3d_a(sq + slot * C::kTileBytes + a * C::kAtomBytes, &tm_q,
-                             BAR(kBarQFull + slot), a * 64, q0, (int)bh);
-          ptx::tma_load_3d_a(sdo + slot * C::kTileBytes + a * C::kAtomBytes, &tm_do,
-                             BAR(kBarQFull + slot), a * 64, q0, (int)bh);
-        }
-      }
+      if (lane == 0) ptx::mbar_arrive_a(BAR(kBarQFull + slot));
       ++n;
+      it = next_live(it + 1);
+      fetch(it);  // in flight while the next buffer frees up
     }
     // drain: the last loads land before the CTA exits
     if (lane == 0) {

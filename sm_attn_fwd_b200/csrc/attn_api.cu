@@ -746,7 +746,8 @@ attn_status_t attn_bwd(const void* q, const void* k, const void* v, const void* 
   if (mask_kind == ATTN_MASK_DRAFT_BLOCK && draft_block < 1) return ATTN_ERR_INVALID_ARG;
   if (doc_ids && (!aligned(doc_ids, 4) || Lq > Lk)) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
-  if ((long long)B * Hkv > kMaxGridY) return ATTN_ERR_UNSUPPORTED;
+  if (ceil_div(Lk, kBlockN) > kMaxGridY || (long long)B * Hkv > 0x7fffffffLL)
+    return ATTN_ERR_UNSUPPORTED;
   const size_t need = attn_bwd_workspace_size(B, Hq, Lq, d);
   if (need == 0 || ws_bytes < need) return ATTN_ERR_WORKSPACE;
 

@@ -8,9 +8,9 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q,
 // and P_ij = exp(S_ij - LSE_i) from the forward's log-sum-exp.
 //
-// B200 mapping.  One CTA per (b, kv head, 128-key tile), 192 threads; it keeps
-// its K and V tiles in shared memory and walks every query tile of every query
-// head of its group:
+// B200 mapping.  One CTA per (b, kv head, 128-key tile), 192 threads, the
+// heaviest key tiles dispatched first; it keeps its K and V tiles in shared
+// memory and walks every query tile of every query head of its group:
 //   warp 0     TMA producer: K and V once; per query tile Q, dO and, by all
 //              lanes, the tile's row statistics (LSE in base 2, D, document ids).
 //   warp 1     tcgen05.mma issue (elect.sync): S^T = K Q^T and dP^T = V dO^T
@@ -182,9 +182,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int k0 = blockIdx.x * 128;
-  const int b = blockIdx.y / p.Hkv;
-  const int hkv = blockIdx.y % p.Hkv;
+  // blockIdx.x: (b, kv head), fastest; blockIdx.y: key tile.  Blocks are
+  // dispatched x-fastest, so every head's key tile 0 (the most query tiles
+  // under a causal or draft mask) goes out first and the light last tiles
+  // fill the tail.
+  const int k0 = blockIdx.y * 128;
+  const int b = blockIdx.x / p.Hkv;
+  const int hkv = blockIdx.x % p.Hkv;
   const int n_iter = p.group * p.q_tiles;  // (query head of the group, query tile)
 
   if (threadIdx.x == 0) {
@@ -618,7 +622,7 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
     return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   });
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)((p.Lk + 127) / 128), (unsigned)(p.B * p.Hkv), 1);
+  const dim3 grid((unsigned)(p.B * p.Hkv), (unsigned)((p.Lk + 127) / 128), 1);
   kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

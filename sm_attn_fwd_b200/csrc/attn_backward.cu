@@ -605,6 +605,477 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// d = 64: the pipelined backward.  Tensor memory has room for P^T of its own
+// ([448, 512)), and dK = dS^T Q reads dS^T from shared memory (the K-major
+// reading of the tile the dQ MMA reads as MN-major), so the score columns are
+// free as soon as the softmax warps have loaded them: S^T and dP^T of the next
+// query tile are computed while the softmax warps still work on this one, and
+// the gradient MMAs of this tile run while they start on the next.  448
+// threads:
+//   warp 0       TMA producer (Q, dO and row statistics in three buffers)
+//   warp 1       MMA issue
+//   warps 2-9    softmax, two warps per TMEM lane quarter, each taking 64 of
+//                the 128 query columns of its keys: P^T to tensor memory,
+//                dS^T to shared memory; at the end dK and dV (32 columns of d
+//                each)
+//   warps 10-13  dQ: read the dQ tile out of tensor memory into the staging
+//                tile, which TMA bulk reduce-adds into the fp32 accumulator
+namespace {
+
+constexpr int kPipeThreads = 448;
+constexpr int kPipeSmThreads = 256;  // softmax threads
+constexpr int kPipeDqIssuer = 320;   // warp 10, lane 0
+
+struct PipeCfg {
+  static constexpr int kQBufs = 3;
+  static constexpr int kAtomBytes = 128 * 128;
+  static constexpr int kTileBytes = 128 * 64 * 2;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kTileBytes;
+  static constexpr int kOffQ = kOffV + kTileBytes;                  // [kQBufs]
+  static constexpr int kOffDO = kOffQ + kQBufs * kTileBytes;        // [kQBufs]
+  static constexpr int kOffDS = kOffDO + kQBufs * kTileBytes;       // dS^T [128 keys][128 queries]
+  static constexpr int kOffStage = kOffDS + 2 * kAtomBytes;         // dQ staging, two boxes
+  static constexpr int kStageBoxBytes = 128 * 128;
+  static constexpr int kStatWords = 400;
+  static constexpr int kOffStat = kOffStage + 2 * kStageBoxBytes;   // [kQBufs] x kStatWords
+  static constexpr int kOffBar = kOffStat + kQBufs * kStatWords * 4;
+  static constexpr int kNumBars = 16;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16;
+  static constexpr int kSmemAlloc = kSmemBytes + 1024;
+  static_assert(kSmemAlloc <= 227 * 1024, "shared memory");
+  // tensor-memory columns
+  static constexpr uint32_t kST = 0, kDPT = 128, kDV = 256, kDK = 320, kDQ = 384, kPT = 448;
+};
+
+enum : int { kPKv = 0, kPQFull = 1, kPQEmpty = 4, kPSFull = 7, kPSFree, kPPFull, kPGradDone,
+             kPDqFree, kPAcc, kPStageFull, kPStageFree };
+
+}  // namespace
+
+__global__ void __launch_bounds__(kPipeThreads, 1)
+    attn_bwd64_pipe_kernel(const __grid_constant__ CUtensorMap tm_q,
+                           const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v,
+                           const __grid_constant__ CUtensorMap tm_do,
+                           const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  using C = PipeCfg;
+  constexpr int QB = C::kQBufs;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sk = ptx::smem_u32(smem + C::kOffK);
+  const uint32_t sv = ptx::smem_u32(smem + C::kOffV);
+  const uint32_t sq = ptx::smem_u32(smem + C::kOffQ);
+  const uint32_t sdo = ptx::smem_u32(smem + C::kOffDO);
+  const uint32_t sds = ptx::smem_u32(smem + C::kOffDS);
+  const uint32_t sstage = ptx::smem_u32(smem + C::kOffStage);
+  float* stat_s = reinterpret_cast<float*>(smem + C::kOffStat);
+  const uint32_t bar0 = ptx::smem_u32(smem + C::kOffBar);
+  auto BAR = [bar0](int i) -> uint32_t { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  int* err = p.err;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // blockIdx.x: (b, kv head), fastest; blockIdx.y: key tile (heaviest first)
+  const int k0 = blockIdx.y * 128;
+  const int b = blockIdx.x / p.Hkv;
+  const int hkv = blockIdx.x % p.Hkv;
+  const int n_iter = p.group * p.q_tiles;  // (query head of the group, query tile)
+
+  if (threadIdx.x == 0) {
+    ptx::prefetch_tmap(&tm_q);
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+    ptx::prefetch_tmap(&tm_do);
+    ptx::prefetch_tmap(&tm_dq);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    ptx::mbar_init(&bars[kPKv], 1);
+    for (int i = 0; i < QB; ++i) {
+      ptx::mbar_init(&bars[kPQFull + i], 1);
+      ptx::mbar_init(&bars[kPQEmpty + i], 1);
+    }
+    ptx::mbar_init(&bars[kPSFull], 1);
+    ptx::mbar_init(&bars[kPSFree], kPipeSmThreads);
+    ptx::mbar_init(&bars[kPPFull], kPipeSmThreads);
+    ptx::mbar_init(&bars[kPGradDone], 1);
+    ptx::mbar_init(&bars[kPDqFree], 128);
+    ptx::mbar_init(&bars[kPAcc], 1);
+    ptx::mbar_init(&bars[kPStageFull], 128);
+    ptx::mbar_init(&bars[kPStageFree], 1);
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kBwdTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  auto iter_q0 = [&](int it) { return (it % p.q_tiles) * 128; };
+  auto iter_hq = [&](int it) { return hkv * p.group + it / p.q_tiles; };
+  auto next_live = [&](int it) {
+    while (it < n_iter && !pair_live(p, k0, iter_q0(it))) ++it;
+    return it;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    bool ok = true;
+    constexpr uint32_t kTx = C::kTileBytes;
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx_a(BAR(kPKv), 2 * kTx);
+      ptx::tma_load_3d_a(sk, &tm_k, BAR(kPKv), 0, k0, b * p.Hkv + hkv);
+      ptx::tma_load_3d_a(sv, &tm_v, BAR(kPKv), 0, k0, b * p.Hkv + hkv);
+    }
+    float f_nl2[4], f_nds[4];
+    int f_doc[4];
+    auto fetch = [&](int it) {
+      const int q0 = iter_q0(it);
+      const long long bh = (long long)b * p.Hq + iter_hq(it);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int qi = q0 + lane + 32 * m;
+        f_nl2[m] = -INFINITY;
+        f_nds[m] = 0.0f;
+        f_doc[m] = 0;
+        if (it < n_iter && qi < p.Lq) {
+          const float lse = __ldg(p.lse + bh * p.Lq + qi);
+          f_nl2[m] = (lse == -INFINITY) ? -INFINITY : -(lse * kLog2eB);
+          f_nds[m] = -__ldg(p.dsum + bh * p.Lq + qi);
+          if (p.doc_ids != nullptr)
+            f_doc[m] = __ldg(p.doc_ids + (long long)b * p.Lk + (p.Lk - p.Lq + qi));
+        }
+      }
+    };
+    int n = 0;
+    int it = next_live(0);
+    fetch(it);
+    while (it < n_iter && ok) {
+      const int q0 = iter_q0(it);
+      const long long bh = (long long)b * p.Hq + iter_hq(it);
+      const int slot = n % QB;
+      if (n >= QB) {
+        ok = ptx::mbar_wait_a(BAR(kPQEmpty + slot), (uint32_t)(n / QB - 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutProducer);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      if (lane == 0) {
+        ptx::mbar_expect_tx_a(BAR(kPQFull + slot), 2 * kTx);
+        ptx::tma_load_3d_a(sq + slot * C::kTileBytes, &tm_q, BAR(kPQFull + slot), 0, q0, (int)bh);
+        ptx::tma_load_3d_a(sdo + slot * C::kTileBytes, &tm_do, BAR(kPQFull + slot), 0, q0,
+                           (int)bh);
+      }
+      float* nl2_s = stat_s + slot * C::kStatWords;
+      float* nds_s = nl2_s + 128;
+      int* qdoc_s = reinterpret_cast<int*>(nds_s + 128);
+      int dmin = 0x7fffffff, dmax = (int)0x80000000;
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int r = lane + 32 * m;
+        nl2_s[r] = f_nl2[m];
+        nds_s[r] = f_nds[m];
+        qdoc_s[r] = f_doc[m];
+        if (q0 + r < p.Lq) {
+          dmin = min(dmin, f_doc[m]);
+          dmax = max(dmax, f_doc[m]);
+        }
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        dmin = min(dmin, __shfl_xor_sync(0xffffffffu, dmin, o));
+        dmax = max(dmax, __shfl_xor_sync(0xffffffffu, dmax, o));
+      }
+      if (lane == 0) {
+        qdoc_s[128] = p.doc_ids != nullptr ? dmin : 0;
+        qdoc_s[129] = p.doc_ids != nullptr ? dmax : 0;
+      }
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_a(BAR(kPQFull + slot));
+      ++n;
+      it = next_live(it + 1);
+      fetch(it);
+    }
+    if (lane == 0) {
+      int dummy = 0;
+      ptx::mbar_wait_a(BAR(kPKv), 0, &dummy, nullptr, 0);
+      for (int jj = max(0, n - QB); jj < n; ++jj) {
+        dummy = 0;
+        ptx::mbar_wait_a(BAR(kPQFull + jj % QB), (uint32_t)(jj / QB) & 1u, &dummy, nullptr, 0);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issue
+    constexpr uint32_t kIdS = ptx::idesc_bf16_f32(128, 128, 0, 0);   // K-major A and B
+    constexpr uint32_t kIdAcc = ptx::idesc_bf16_f32(128, 64, 0, 1);  // A K-major / TMEM, B MN
+    constexpr uint32_t kIdDq = ptx::idesc_bf16_f32(128, 64, 1, 1);   // A and B MN-major
+    bool ok = ptx::mbar_wait_a(BAR(kPKv), 0, abort_flag, err, kDevErrTimeoutMma);
+    ok = __all_sync(0xffffffffu, ok);
+    int it = next_live(0);
+    auto issue_scores = [&](int n) -> bool {
+      const int slot = n % QB;
+      bool good = ptx::mbar_wait_a(BAR(kPQFull + slot), (uint32_t)(n / QB) & 1u, abort_flag, err,
+                                   kDevErrTimeoutMma);
+      good = __all_sync(0xffffffffu, good);
+      if (!good) return false;
+      ptx::tc_fence_after();
+      ptx::mma_qk_chain_d64(tmem + C::kST, bdesc(sk, 16), bdesc(sq + slot * C::kTileBytes, 16),
+                            kIdS);
+      ptx::mma_qk_chain_d64(tmem + C::kDPT, bdesc(sv, 16), bdesc(sdo + slot * C::kTileBytes, 16),
+                            kIdS);
+      ptx::mma_commit_warp(BAR(kPSFull));
+      return true;
+    };
+    if (ok && it < n_iter) ok = issue_scores(0);
+    int n = 0;
+    while (ok && it < n_iter) {
+      const int it_next = next_live(it + 1);
+      const int slot = n % QB;
+      const uint32_t sq_n = sq + slot * C::kTileBytes, sdo_n = sdo + slot * C::kTileBytes;
+      if (it_next < n_iter) {
+        // the next tile's scores, once the softmax warps hold this tile's in registers
+        ok = ptx::mbar_wait_a(BAR(kPSFree), (uint32_t)n & 1u, abort_flag, err, kDevErrTimeoutMma);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        ok = issue_scores(n + 1);
+        if (!ok) break;
+      }
+      ok = ptx::mbar_wait_a(BAR(kPPFull), (uint32_t)n & 1u, abort_flag, err, kDevErrTimeoutMma);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const uint32_t acc = n > 0 ? 1u : 0u;
+      // dV += P^T dO (P^T from tensor memory)
+      ptx::mma_pv_chain8(tmem + C::kDV, tmem + C::kPT, bdesc(sdo_n, C::kAtomBytes), kIdAcc, acc);
+      // dK += dS^T Q (dS^T K-major from shared memory: 64 queries per atom)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        ptx::mma_ss_warp(tmem + C::kDK,
+                         bdesc(sds + (uint32_t)((kk >> 2) * C::kAtomBytes + (kk & 3) * 32), 16),
+                         bdesc(sq_n + (uint32_t)(kk * 2048), C::kAtomBytes), kIdAcc,
+                         (n > 0 || kk > 0) ? 1u : 0u);
+      if (n > 0) {  // the previous dQ tile has been read out
+        ok = ptx::mbar_wait_a(BAR(kPDqFree), (uint32_t)(n - 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutMma);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        ptx::tc_fence_after();
+      }
+      // dQ_tile = dS K
+      mma_ss_chain8_mn(tmem + C::kDQ, bdesc(sds, C::kAtomBytes), bdesc(sk, C::kAtomBytes), kIdDq);
+      ptx::mma_commit_warp(BAR(kPQEmpty + slot));
+      ptx::mma_commit_warp(BAR(kPGradDone));
+      ++n;
+      it = it_next;
+    }
+    ptx::mma_commit_warp(BAR(kPAcc));
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;        // query columns [64 half, 64 half + 64)
+    const int row = quarter * 32 + lane;     // key of the tile (TMEM lane)
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int key = k0 + row;
+    int qlo = 0, qhi = -1;
+    if (key < p.Lk) query_bounds(p, key, qlo, qhi);
+    const int kdoc = (p.doc_ids != nullptr && key < p.Lk)
+                         ? __ldg(p.doc_ids + (long long)b * p.Lk + key) : 0;
+    const float c = p.scale_log2;
+    bool ok = true;
+    int n = 0;
+    for (int it = next_live(0); it < n_iter && ok; it = next_live(it + 1)) {
+      const int q0 = iter_q0(it);
+      const uint32_t stats = ptx::smem_u32(stat_s + (n % QB) * C::kStatWords);
+      const int* qdoc_s = reinterpret_cast<const int*>(stat_s + (n % QB) * C::kStatWords + 256);
+      ok = ptx::mbar_wait_a(BAR(kPSFull), (uint32_t)n & 1u, abort_flag, err,
+                            kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      bool sees_all = key < p.Lk && qlo <= q0 && qhi >= q0 + 127;
+      if (p.doc_ids != nullptr) sees_all = sees_all && qdoc_s[128] == kdoc && qdoc_s[129] == kdoc;
+      const bool full = __all_sync(0xffffffffu, sees_all);
+#pragma unroll 1
+      for (int j = 0; j < 2 && ok; ++j) {
+        const int cc = 2 * half + j;  // 32 query columns
+        uint32_t rs[32], rd[32];
+        ptx::tmem_ld32(t_row + C::kST + cc * 32, rs);
+        ptx::tmem_ld32(t_row + C::kDPT + cc * 32, rd);
+        ptx::tmem_wait_ld();
+        if (j == 1) {  // every score column of this tile is in registers
+          ptx::tc_fence_before();
+          ptx::mbar_arrive_a(BAR(kPSFree));
+        }
+        uint32_t pp[16], dp[16];
+#pragma unroll
+        for (int g4 = 0; g4 < 8; ++g4) {  // four query columns per step
+          uint32_t w0, w1, w2, w3;
+          float nl[4], nd[4];
+          ptx::ld_shared_v4(stats + (uint32_t)(cc * 128 + g4 * 16), w0, w1, w2, w3);
+          nl[0] = __uint_as_float(w0);
+          nl[1] = __uint_as_float(w1);
+          nl[2] = __uint_as_float(w2);
+          nl[3] = __uint_as_float(w3);
+          ptx::ld_shared_v4(stats + (uint32_t)(512 + cc * 128 + g4 * 16), w0, w1, w2, w3);
+          nd[0] = __uint_as_float(w0);
+          nd[1] = __uint_as_float(w1);
+          nd[2] = __uint_as_float(w2);
+          nd[3] = __uint_as_float(w3);
+          if (!full) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int col = cc * 32 + 4 * g4 + i;
+              bool vis = q0 + col >= qlo && q0 + col <= qhi;
+              if (p.doc_ids != nullptr) vis = vis && (qdoc_s[col] == kdoc);
+              nl[i] = vis ? nl[i] : -INFINITY;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 4; i += 2) {
+            const int e = 4 * g4 + i;
+            float x0, x1, d0, d1;
+            ptx::fma2_bv(x0, x1, __uint_as_float(rs[e]), __uint_as_float(rs[e + 1]), c, nl[i],
+                         nl[i + 1]);
+            const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+            ptx::addmul2(d0, d1, __uint_as_float(rd[e]), __uint_as_float(rd[e + 1]), nd[i],
+                         nd[i + 1], p0, p1);
+            pp[e / 2] = ptx::pack_bf16x2(p0, p1);
+            dp[e / 2] = ptx::pack_bf16x2(d0, d1);
+          }
+        }
+        if (j == 0 && n > 0) {  // P^T and dS^T of the previous tile have been used
+          ok = ptx::mbar_wait_a(BAR(kPGradDone), (uint32_t)(n - 1) & 1u, abort_flag, err,
+                                kDevErrTimeoutSoftmax);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          ptx::tc_fence_after();
+        }
+        ptx::tmem_st16(t_row + C::kPT + cc * 16, pp);
+        const uint32_t atom = sds + (uint32_t)((cc >> 1) * C::kAtomBytes) + (uint32_t)row * 128u;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const uint32_t chunk = (uint32_t)((cc & 1) * 4 + q4);
+          const uint32_t addr = atom + ((chunk ^ (uint32_t)(row & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(dp[4 * q4]),
+                       "r"(dp[4 * q4 + 1]), "r"(dp[4 * q4 + 2]), "r"(dp[4 * q4 + 3])
+                       : "memory");
+        }
+      }
+      if (!ok) break;
+      ptx::tmem_wait_st();
+      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_a(BAR(kPPFull));
+      ++n;
+    }
+    // dK (times scale) and dV: 32 columns of d per half
+    if (ok) {
+      ok = ptx::mbar_wait_a(BAR(kPAcc), 0, abort_flag, err, kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    ptx::tc_fence_after();
+    const long long base = (((long long)b * p.Hkv + hkv) * p.Lk + key) * 64 + half * 32;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(which ? p.dv : p.dk) + base;
+      const float f = which ? 1.0f : p.scale;
+      uint32_t r[32];
+      if (ok && n > 0) {  // warp-uniform
+        ptx::tmem_ld32(t_row + (which ? C::kDV : C::kDK) + (uint32_t)(half * 32), r);
+        ptx::tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = 0u;
+      }
+      if (key < p.Lk) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          uint4 v4;
+          v4.x = ptx::pack_bf16x2(__uint_as_float(r[i]) * f, __uint_as_float(r[i + 1]) * f);
+          v4.y = ptx::pack_bf16x2(__uint_as_float(r[i + 2]) * f, __uint_as_float(r[i + 3]) * f);
+          v4.z = ptx::pack_bf16x2(__uint_as_float(r[i + 4]) * f, __uint_as_float(r[i + 5]) * f);
+          v4.w = ptx::pack_bf16x2(__uint_as_float(r[i + 6]) * f, __uint_as_float(r[i + 7]) * f);
+          *reinterpret_cast<uint4*>(out + i) = v4;
+        }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------------- dQ
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // query of the tile (TMEM lane)
+    const uint32_t t_row = tmem + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    int n = 0;
+    for (int it = next_live(0); it < n_iter && ok; it = next_live(it + 1)) {
+      const int q0 = iter_q0(it);
+      const long long bh = (long long)b * p.Hq + iter_hq(it);
+      ok = ptx::mbar_wait_a(BAR(kPGradDone), (uint32_t)n & 1u, abort_flag, err,
+                            kDevErrTimeoutSoftmax);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (n > 0) {  // the staging tile has been read by the previous reduce
+        if (threadIdx.x == kPipeDqIssuer) {
+          ptx::bulk_wait_group_read0();
+          ptx::mbar_arrive_a(BAR(kPStageFree));
+        }
+        ok = ptx::mbar_wait_a(BAR(kPStageFree), (uint32_t)(n - 1) & 1u, abort_flag, err,
+                              kDevErrTimeoutSoftmax);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+      }
+      uint32_t r[2][32];
+      ptx::tmem_ld32(t_row + C::kDQ, r[0]);
+      ptx::tmem_ld32(t_row + C::kDQ + 32, r[1]);
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_a(BAR(kPDqFree));
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const uint32_t rowp = sstage + (uint32_t)(c2 * C::kStageBoxBytes) + (uint32_t)row * 128u;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint32_t addr = rowp + (((uint32_t)ch ^ (uint32_t)(row & 7)) << 4);
+          asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                       "f"(__uint_as_float(r[c2][4 * ch]) * p.scale),
+                       "f"(__uint_as_float(r[c2][4 * ch + 1]) * p.scale),
+                       "f"(__uint_as_float(r[c2][4 * ch + 2]) * p.scale),
+                       "f"(__uint_as_float(r[c2][4 * ch + 3]) * p.scale)
+                       : "memory");
+        }
+      }
+      ptx::fence_proxy_async_smem();
+      ptx::mbar_arrive_a(BAR(kPStageFull));
+      if (threadIdx.x == kPipeDqIssuer) {
+        ok = ptx::mbar_wait_a(BAR(kPStageFull), (uint32_t)n & 1u, abort_flag, err,
+                              kDevErrTimeoutSoftmax);
+        if (ok) {
+          ptx::tma_reduce_add_3d(&tm_dq, sstage, 0, q0, (int)bh);
+          ptx::tma_reduce_add_3d(&tm_dq, sstage + C::kStageBoxBytes, 32, q0, (int)bh);
+          ptx::bulk_commit_group();
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      ++n;
+    }
+    if (threadIdx.x == kPipeDqIssuer) ptx::bulk_wait_group0();
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kBwdTmemCols);
+  }
+}
+
 // The three launches of the backward: D_i, the main kernel, dQ to bf16.  The
 // caller zeroes dq_acc before (on the same stream).
 template <int D>
@@ -615,15 +1086,26 @@ cudaError_t launch_backward(const CUtensorMap& tq, const CUtensorMap& tk, const 
   attn_bwd_dsum_kernel<D><<<(unsigned)((nrows + 7) / 8), 256, 0, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  auto kern = attn_bwd_kernel<D>;
-  constexpr int smem = BwdCfg<D>::kSmemAlloc;
-  static PerContextOnce once;
-  e = once_per_context(once, [&](int) {
-    return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  });
-  if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)(p.B * p.Hkv), (unsigned)((p.Lk + 127) / 128), 1);
-  kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, p);
+  if constexpr (D == 64) {
+    constexpr int smem = PipeCfg::kSmemAlloc;
+    static PerContextOnce once;
+    e = once_per_context(once, [&](int) {
+      return cudaFuncSetAttribute(attn_bwd64_pipe_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (e != cudaSuccess) return e;
+    attn_bwd64_pipe_kernel<<<grid, kPipeThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, p);
+  } else {
+    auto kern = attn_bwd_kernel<D>;
+    constexpr int smem = BwdCfg<D>::kSmemAlloc;
+    static PerContextOnce once;
+    e = once_per_context(once, [&](int) {
+      return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    });
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kBwdThreads, smem, stream>>>(tq, tk, tv, tdo, tdq, p);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long n4 = nrows * D / 4;

@@ -534,12 +534,15 @@ def main():
                     help="with --only: set the batch size B (smaller profiling case)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="with --only on a prefill workload: Lq = Lk = this length (profiling)")
+    ap.add_argument("--head-dim", type=int, default=None,
+                    help="with --only on a prefill workload: this head dimension (profiling)")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="--impl reference: total CPU seconds across all steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
-                    help="also time attn_bwd on the headline workload (reported under workloads)")
+                    help="also time attn_bwd on the headline workload (reported under workloads);"
+                         " with --only, time attn_bwd on that workload instead of the forward")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" and args.only is None else args.warmup
 
@@ -563,7 +566,13 @@ def main():
             cfg = cfg.with_(B=args.batch, name=f"{cfg.name}_B{args.batch}")
         if args.seq_len is not None and not cfg.decode:
             cfg = cfg.with_(Lq=args.seq_len, Lk=args.seq_len, name=f"{cfg.name}_L{args.seq_len}")
-        if cfg.decode:
+        if args.head_dim is not None and not cfg.decode:
+            cfg = cfg.with_(d=args.head_dim, name=f"{cfg.name}_d{args.head_dim}")
+        if args.backward and not cfg.decode:
+            ms, flops = run_backward(cfg, timer, args.steps, args.warmup, stream)
+            print(json.dumps({"workload": cfg.name + "_backward", "ms": ms,
+                              "TFLOP/s": flops / (statistics.median(ms) * 1e9)}))
+        elif cfg.decode:
             _, ms, nbytes, plan = run_decode(cfg, timer, args.steps, args.warmup, stream)
             print(json.dumps({"workload": cfg.name, "ms": ms, "GB/s": nbytes / (statistics.median(ms) * 1e6)}))
         else:

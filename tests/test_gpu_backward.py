@@ -71,3 +71,30 @@ def test_backward_rejects_on_host():
     with pytest.raises(ab.AttnError) as e:
         ab.attn_bwd(q, q, q, q, lse, q)               # d = 96 not built
     assert e.value.status == ab.ATTN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_backward_full_size_sampled_heads(d):
+    """The benchmark's backward workload (causal, B=2, H=16, L=4096, d=64, and the
+    same at d=128) on the inputs and dO the benchmark draws: whole heads of dQ,
+    dK and dV compared with the oracle run on those heads alone (heads are
+    independent without GQA)."""
+    from workloads import CAUSAL_4K, make_inputs
+    cfg = CAUSAL_4K.with_(d=d)
+    inp = make_inputs(cfg)
+    g = torch.Generator()
+    g.manual_seed(cfg.seed + 1000)
+    do = torch.randn(inp.q.shape, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = to_dev(inp.q, inp.k, inp.v, do)
+    o, lse = ab.attn_fwd(qd, kd, vd, scale=cfg.softmax_scale, mask="causal")
+    dq, dk, dv = ab.attn_bwd(qd, kd, vd, o, lse, dod, scale=cfg.softmax_scale, mask="causal")
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    for b, h in ((0, 3), (1, 15)):
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        rq, rk, rv = oracle.attn_bwd(inp.q[sl], inp.k[sl], inp.v[sl], do[sl],
+                                     scale=cfg.softmax_scale, mask="causal")
+        _check(dv[sl], rv, f"dV b{b} h{h} d{d}")
+        _check(dk[sl], rk, f"dK b{b} h{h} d{d}")
+        _check(dq[sl], rq, f"dQ b{b} h{h} d{d}")

@@ -98,3 +98,30 @@ def test_backward_full_size_sampled_heads(d):
         _check(dv[sl], rv, f"dV b{b} h{h} d{d}")
         _check(dk[sl], rk, f"dK b{b} h{h} d{d}")
         _check(dq[sl], rq, f"dQ b{b} h{h} d{d}")
+
+
+def test_backward_capturable_in_cuda_graph():
+    """attn_bwd (memset, D_i kernel, gradient kernel, dQ conversion) replays from
+    a CUDA graph with the results of a direct call."""
+    q, k, v, _, _ = random_case(31, 1, 4, 2, 300, 300, 64)
+    do = torch.randn(1, 4, 300, 64, generator=torch.Generator().manual_seed(131)).to(torch.bfloat16)
+    qd, kd, vd, dod = to_dev(q, k, v, do)
+    o, lse = ab.attn_fwd(qd, kd, vd, mask="causal")
+    ws = torch.empty(ab.load_library().attn_bwd_workspace_size(1, 4, 300, 64), dtype=torch.uint8,
+                     device="cuda")
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
+    s = torch.cuda.Stream()
+    kw = dict(mask="causal", workspace=ws, dq=dq, dk=dk, dv=dv, stream=s)
+    with torch.cuda.stream(s):
+        ab.attn_bwd(qd, kd, vd, o, lse, dod, **kw)           # set-up outside the capture
+    s.synchronize()
+    ref = (dq.clone(), dk.clone(), dv.clone())
+    g = torch.cuda.CUDAGraph()
+    dq.zero_(); dk.zero_(); dv.zero_()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        ab.attn_bwd(qd, kd, vd, o, lse, dod, **kw)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+    _check(dq, ref[0].float().cpu().double().numpy(), "dQ graph replay")

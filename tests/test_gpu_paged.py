@@ -92,3 +92,38 @@ def test_bad_page_id_is_flagged_not_faulted():
     st, bits = ab.attn_get_device_error()
     assert st == ab.ATTN_ERR_INVALID_ARG and bits != 0
     assert ab.attn_get_device_error()[0] == ab.ATTN_OK
+
+
+def test_bench_paged_workloads_equal_contiguous():
+    """The benchmark's paged legs: the full Lq=1 decode cache (B=64, Hq=64, Hkv=8,
+    32K keys, d=128) moved into a shuffled page pool of 128- and of 16-key pages
+    exactly as the benchmark does; the paged call gives the contiguous call's O
+    and LSE to the bit (the contiguous call is checked against the oracle in the
+    full-size decode test)."""
+    from workloads import DECODE_LQ1, make_inputs
+    cfg = DECODE_LQ1
+    inp = make_inputs(cfg, device="cuda")
+    o_c, l_c = ab.attn_decode_splitkv(inp.q, inp.k, inp.v, inp.kv_lens, scale=cfg.softmax_scale)
+    B, Hkv, L, d = inp.k.shape
+    for page_size in (128, 16):
+        pps = L // page_size
+        g = torch.Generator(device="cuda")
+        g.manual_seed(cfg.seed + 1000)
+        perm = torch.randperm(B * pps, generator=g, device="cuda")
+
+        def to_pool(x):
+            pages = x.view(B, Hkv, pps, page_size, d).permute(0, 2, 1, 3, 4).reshape(
+                B * pps, Hkv, page_size, d)
+            pool = torch.empty_like(pages)
+            pool[perm] = pages
+            return pool
+        kp, vp = to_pool(inp.k), to_pool(inp.v)
+        table = perm.view(B, pps).to(torch.int32).contiguous()
+        o_p, l_p = ab.attn_decode_paged(inp.q, kp, vp, table, inp.kv_lens,
+                                        scale=cfg.softmax_scale)
+        torch.cuda.synchronize()
+        st, bits = ab.attn_get_device_error()
+        assert st == ab.ATTN_OK, (st, bits)
+        assert torch.equal(o_p, o_c) and torch.equal(l_p, l_c), page_size
+        del kp, vp
+        torch.cuda.empty_cache()

@@ -143,3 +143,23 @@ def test_constant_table_matches_plain_forward():
     assert (o1.float() - o2.float()).abs().max().item() <= 2e-2
     shift = (l1 - l2).cpu()
     assert (shift - consts.view(1, 4, 1)).abs().max().item() <= 1e-3
+
+
+def test_alibi_bench_workload_sampled_rows():
+    """The benchmark's ALiBi leg: the causal 4K workload (B=2, H=16, d=64) with
+    slopes 2^(-8 (h+1) / H), sampled rows against the oracle."""
+    from workloads import CAUSAL_4K, make_inputs
+    cfg = CAUSAL_4K
+    inp = make_inputs(cfg)
+    sl = slopes_for(cfg.Hq)
+    qd, kd, vd = to_dev(inp.q, inp.k, inp.v)
+    o, lse = ab.attn_fwd_score_mod(qd, kd, vd, alibi_slopes=sl.cuda(), scale=cfg.softmax_scale,
+                                   mask="causal")
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    rows = sample_rows(cfg.B, cfg.Hq, cfg.Lq, 64, seed=7)
+    ro, rl = oracle.attn_fwd(inp.q, inp.k, inp.v, scale=cfg.softmax_scale, mask="causal",
+                             rows=rows, alibi_slopes=sl.double().numpy())
+    idx = torch.from_numpy(rows).cuda()
+    compare(o.reshape(-1, cfg.d)[idx], lse.reshape(-1)[idx], ro, rl, "alibi bench workload")

@@ -104,3 +104,23 @@ def test_bad_cu_seqlens_flagged_and_skipped():
     assert st == ab.ATTN_ERR_INVALID_ARG
     st, bits = ab.attn_get_device_error()
     assert st == ab.ATTN_OK and bits == 0
+
+
+def test_bench_packed_workload_sampled_sequences():
+    """The benchmark's packed workload (16 causal sequences of 128-4096 tokens,
+    H=16, d=64, seed 5) in one call; the longest, the shortest and two more
+    sequences checked whole against the oracle."""
+    from workloads import packed_case, packed_lengths
+    lens = packed_lengths(5, 16, 128, 4096)
+    q, k, v, cu_q, cu_k = packed_case(5, lens, lens, 16, 16, 64)
+    qd, kd, vd, cqd, ckd = (t.cuda() for t in (q, k, v, cu_q, cu_k))
+    o, lse = ab.attn_fwd_varlen(qd, kd, vd, cqd, ckd, max(lens), mask="causal")
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    order = sorted(range(16), key=lambda i: lens[i])
+    for b in sorted({order[0], order[-1], order[5], order[10]}):
+        t0, t1 = int(cu_q[b]), int(cu_q[b + 1])
+        one = torch.tensor([0, t1 - t0], dtype=torch.int32)
+        ro, rl = oracle.attn_fwd_varlen(q[t0:t1], k[t0:t1], v[t0:t1], one, one, mask="causal")
+        compare(o[t0:t1], lse[:, t0:t1], ro, rl, f"sequence {b}")

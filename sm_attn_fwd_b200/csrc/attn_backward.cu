@@ -8,11 +8,15 @@
 //   dQ = scale * dS K,  dK = scale * dS^T Q,
 // and P_ij = exp(S_ij - LSE_i) from the forward's log-sum-exp.
 //
-// B200 mapping.  One CTA per (b, kv head, 128-key tile), 192 threads, the
-// heaviest key tiles dispatched first; it keeps its K and V tiles in shared
-// memory and walks every query tile of every query head of its group:
+// B200 mapping.  Two gradient kernels: attn_bwd64_pipe_kernel (d = 64, below,
+// with its own description) and attn_bwd_kernel<D>, which the library runs for
+// d = 128.  attn_bwd_kernel: one CTA per (b, kv head, 128-key tile), 192
+// threads, the heaviest key tiles dispatched first; it keeps its K and V tiles
+// in shared memory and walks every query tile of every query head of its
+// group:
 //   warp 0     TMA producer: K and V once; per query tile Q, dO and, by all
-//              lanes, the tile's row statistics (LSE in base 2, D, document ids).
+//              lanes, the tile's row statistics (-LSE in base 2, -D, document
+//              ids), loaded one tile ahead.
 //   warp 1     tcgen05.mma issue (elect.sync): S^T = K Q^T and dP^T = V dO^T
 //              (both operands K-major in shared memory), then dV += P^T dO and
 //              dK += dS^T Q (P^T, dS^T from tensor memory, dO, Q MN-major), and
@@ -20,17 +24,15 @@
 //   warps 2-5  one key per thread (its TMEM lane): P^T and dS^T for 128 query
 //              columns, written to tensor memory (bf16, over S^T and dP^T) and
 //              dS^T to shared memory; then, one query per thread, the dQ tile
-//              is reduced into an fp32 accumulator in global memory; at the end
-//              dK (times scale) and dV are stored as bf16.
-// Tensor memory (512 columns).  d = 64: S^T / P^T [0,128), dP^T / dS^T
-// [128,256), dV [256,320), dK [320,384), dQ tile [384,448).  d = 128: dV
-// [256,384), dK [384,512); P^T and dS^T (bf16) take the lower 64 columns of
-// S^T and dP^T, and the dQ tile (fp32, 128 columns) is computed as two
-// 64-column halves into the freed upper halves, [64,128) and [192,256).
-// With d = 64, Q, dO and the row statistics are double-buffered: the next
-// query tile's loads, S^T and dP^T run while the softmax warps reduce this
-// tile's dQ.  (With d = 128 the second buffers do not fit in shared memory,
-// and S^T of the next tile must wait for the dQ read-out anyway.)
+//              is staged in shared memory and added into an fp32 accumulator in
+//              global memory by TMA reduce-adds; at the end dK (times scale)
+//              and dV are stored as bf16.
+// Tensor memory (512 columns) at d = 128: dV [256,384), dK [384,512); P^T and
+// dS^T (bf16) take the lower 64 columns of S^T [0,128) and dP^T [128,256), and
+// the dQ tile (fp32, 128 columns) is computed as two 64-column halves into the
+// freed upper halves, [64,128) and [192,256), so S^T of the next query tile
+// waits for the dQ read-out; Q, dO and the row statistics have one buffer (a
+// second does not fit in shared memory).
 // Small kernels before and after: D_i, and dQ from its fp32 accumulator.
 #include <cuda.h>
 #include <cuda_bf16.h>

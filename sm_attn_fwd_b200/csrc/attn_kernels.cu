@@ -48,6 +48,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kCopyWarps = 3;
 constexpr int kTmemCols = 512;
+static_assert(kBlockN == 128, "the softmax handles 128-key tiles");
 constexpr uint32_t kTmemO = 256;
 // S (and P over it) double buffer: columns [0,128) and [128,256).
 __device__ __forceinline__ uint32_t tmem_s(int j) { return (j & 1) ? 128u : 0u; }
@@ -409,26 +410,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
 
       float s[kBlockN];
-      {
-        uint32_t raw[32];
-#pragma unroll
-        for (int cc = 0; cc < kBlockN / 32; ++cc) {
-          ptx::tmem_ld32(t_row + tmem_s(j) + cc * 32, raw);
-          ptx::tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(raw[i]);
-        }
-      }
+      ptx::tmem_ld_row128(t_row + tmem_s(j), s);
       if (!full) {
+        // visible keys of this row inside the tile: [0, hi_rel]
+        const int hi_rel = (int)max(-1LL, min((long long)kBlockN - 1, row_hi - k0));
 #pragma unroll
-        for (int i = 0; i < kBlockN; ++i) {
-          s[i] = (k0 + i <= row_hi) ? s[i] : -INFINITY;
-        }
+        for (int i = 0; i < kBlockN; ++i) s[i] = (i <= hi_rel) ? s[i] : -INFINITY;
       }
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < kBlockN; ++i) mx = fmaxf(mx, s[i]);
-      const float m_tile = mx * c;
+      const float m_tile = ptx::row_max128(s) * c;
       const float m_new = fmaxf(m_ref, m_tile);
       const bool need = m_new > m_ref + kRescaleThreshold;
       const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;  // 0 when m_ref = -inf
@@ -454,20 +443,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = m_new;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      float rowsum = 0.0f;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t packed[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ptx::ex2(fmaf(s[h * 64 + 2 * i], c, -m_use));
-          const float p1 = ptx::ex2(fmaf(s[h * 64 + 2 * i + 1], c, -m_use));
-          rowsum += p0 + p1;
-          packed[i] = ptx::pack_bf16x2(p0, p1);
-        }
-        ptx::tmem_st32(t_row + tmem_s(j) + h * 32, packed);
+      {
+        // P over S: 64 columns of bf16 pairs
+        uint32_t pk_lo[32], pk_hi[32];
+        l += ptx::exp2_pack128(s, c, m_use, pk_lo, pk_hi);
+        ptx::tmem_st32(t_row + tmem_s(j), pk_lo);
+        ptx::tmem_st32(t_row + tmem_s(j) + 32, pk_hi);
       }
-      l += rowsum;
       {
         // Keys past the end of this sequence: their V rows may hold anything
         // (even NaN), and 0 * NaN would poison O.  Zero them in shared memory.

@@ -404,16 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         float s[kBlockN];
-        {
-          uint32_t raw[32];
-#pragma unroll
-          for (int cc = 0; cc < kBlockN / 32; ++cc) {
-            ptx::tmem_ld32(t_row + tmem_s(j) + cc * 32, raw);
-            ptx::tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(raw[i]);
-          }
-        }
+        ptx::tmem_ld_row128(t_row + tmem_s(j), s);
         if (!full) {
 #pragma unroll
           for (int i = 0; i < kBlockN; ++i)
@@ -445,20 +436,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_ref = m_new;
         }
         const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-        float rowsum = 0.0f;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t packed[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const float p0 = ptx::ex2(fmaf(s[h * 64 + 2 * i], c, -m_use));
-            const float p1 = ptx::ex2(fmaf(s[h * 64 + 2 * i + 1], c, -m_use));
-            rowsum += p0 + p1;
-            packed[i] = ptx::pack_bf16x2(p0, p1);
-          }
-          ptx::tmem_st32(t_row + tmem_s(j) + h * 32, packed);
+        {
+          // P over S: 64 columns of bf16 pairs
+          uint32_t pk_lo[32], pk_hi[32];
+          l += ptx::exp2_pack128(s, c, m_use, pk_lo, pk_hi);
+          ptx::tmem_st32(t_row + tmem_s(j), pk_lo);
+          ptx::tmem_st32(t_row + tmem_s(j) + 32, pk_hi);
         }
-        l += rowsum;
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
       }

@@ -69,6 +69,10 @@ def _load():
                                                      i32, i32, i32, i32, P, P, i32, P, i64, P, P,
                                                      i32]
             lib.oracle_attn_rows_relbias.restype = i32
+            lib.oracle_attn_rows_mod.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, f64, i32,
+                                                 i32, i32, i32, P, P, P, P, i32, P, i64, P, P,
+                                                 i32]
+            lib.oracle_attn_rows_mod.restype = i32
             lib.oracle_decode_partials.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f64,
                                                    i32, i32, P, P, i32]
             lib.oracle_decode_partials.restype = i32
@@ -151,9 +155,10 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
     q: [B, Hq, Lq, d] bf16; k, v: [B, Hkv, Lk, d] bf16.  Returns (O, LSE) as
     float64 numpy arrays, shaped [B, Hq, Lq, d] / [B, Hq, Lq], or [n, d] / [n]
     when ``rows`` (flat indices (b*Hq + hq)*Lq + i) is given.  Score modifiers
-    (not with kv_lens): ``alibi_slopes`` ([Hq]) adds slope_h * (j - p) to every
+    (at most one): ``alibi_slopes`` ([Hq]) adds slope_h * (j - p) to every
     scaled score; ``rel_bias`` = (table [Hq, 2R + 1], R) adds
-    table[h, clamp(j - p, -R, R) + R].
+    table[h, clamp(j - p, -R, R) + R]; p = Lk_b - Lq + i, Lk_b = kv_lens[b] when
+    kv_lens is given (the split-KV decode), else Lk.
     """
     qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
     B, Hq, Lq, d = qb.shape
@@ -171,9 +176,31 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
         n = B * Hq * Lq
     o = np.zeros((n, d), dtype=np.float64)
     lse = np.zeros((n,), dtype=np.float64)
-    if rel_bias is not None:
-        if kl is not None or alibi_slopes is not None:
-            raise ValueError("rel_bias is not combined with kv_lens or alibi_slopes")
+    if kl is not None and (rel_bias is not None or alibi_slopes is not None):
+        if rel_bias is not None and alibi_slopes is not None:
+            raise ValueError("rel_bias is not combined with alibi_slopes")
+        sl = tb = None
+        rmax = 0
+        if alibi_slopes is not None:
+            sl = np.ascontiguousarray(np.asarray(
+                alibi_slopes.cpu().numpy() if hasattr(alibi_slopes, "cpu") else alibi_slopes,
+                dtype=np.float64).reshape(-1))
+            if sl.size != Hq:
+                raise ValueError("alibi_slopes must have Hq entries")
+        else:
+            table, rmax = rel_bias
+            tb = np.ascontiguousarray(np.asarray(
+                table.cpu().numpy() if hasattr(table, "cpu") else table, dtype=np.float64))
+            if tb.shape != (Hq, 2 * int(rmax) + 1):
+                raise ValueError("rel_bias table must be [Hq, 2R + 1]")
+        rc = _load().oracle_attn_rows_mod(_ptr(qb), _ptr(kb), _ptr(vb), B, Hq, Hkv, Lq, Lk, d,
+                                          float(scale), _mask_code(mask), int(window[0]),
+                                          int(window[1]), int(draft_block), _ptr(doc), _ptr(kl),
+                                          _ptr(sl), _ptr(tb), int(rmax), _ptr(rows), n, _ptr(o),
+                                          _ptr(lse), int(nthreads or max_threads()))
+    elif rel_bias is not None:
+        if alibi_slopes is not None:
+            raise ValueError("rel_bias is not combined with alibi_slopes")
         table, rmax = rel_bias
         tb = np.ascontiguousarray(np.asarray(
             table.cpu().numpy() if hasattr(table, "cpu") else table, dtype=np.float64))
@@ -185,8 +212,6 @@ def attn_fwd(q, k, v, *, scale=None, mask="none", window=(-1, -1), draft_block=1
                                               _ptr(tb), int(rmax), _ptr(rows), n, _ptr(o),
                                               _ptr(lse), int(nthreads or max_threads()))
     elif alibi_slopes is not None:
-        if kl is not None:
-            raise ValueError("alibi_slopes is not combined with kv_lens")
         sl = np.ascontiguousarray(np.asarray(
             alibi_slopes.cpu().numpy() if hasattr(alibi_slopes, "cpu") else alibi_slopes,
             dtype=np.float64).reshape(-1))

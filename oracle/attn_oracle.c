@@ -315,6 +315,23 @@ int oracle_attn_rows_relbias(const uint16_t* q, const uint16_t* k, const uint16_
                    nthreads);
 }
 
+/* The same with per-sequence key counts kv_lens [B] (may be NULL) and either
+   score modifier (alibi_slopes [Hq] or table [Hq][2 rel_max + 1]; at most one):
+   the split-KV decode with a score_mod, query row i of sequence b at
+   p = kv_lens[b] - Lq + i. */
+int oracle_attn_rows_mod(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                         int Hkv, int Lq, int Lk, int d, double scale, int mask_kind,
+                         int window_l, int window_r, int draft_block, const int32_t* doc_ids,
+                         const int32_t* kv_lens, const double* alibi_slopes, const double* table,
+                         int rel_max, const int64_t* rows, int64_t nrows, double* o, double* lse,
+                         int nthreads) {
+  if (alibi_slopes && table) return -1;
+  if (table && rel_max < 0) return -1;
+  return attn_rows(q, k, v, B, Hq, Hkv, Lq, Lk, d, scale, mask_kind, window_l, window_r,
+                   draft_block, doc_ids, kv_lens, alibi_slopes, table, table ? rel_max : 0, rows,
+                   nrows, o, lse, nthreads);
+}
+
 /*
  * Split-KV decode, step 1 (FlexDecoding / FlashDecoding style split-KV, "FlexAttention
  * 是什么，以及 DFlash2 之谜的完整侦破", section 1): the keys of sequence b,

@@ -311,6 +311,28 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
                                   void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * attn_decode_splitkv_score_mod — attn_decode_splitkv with a score modifier, as
+ * in attn_fwd_score_mod ("FlexAttention 是什么，以及 DFlash2 之谜的完整侦破",
+ * section 1: score_mod(score, b, h, q_idx, kv_idx)).  Query row i of sequence b
+ * sits at absolute position p = kv_lens[b] - Lq + i (the Lq queries are the
+ * last Lq positions of the sequence, the alignment the masks of attn_fwd use):
+ *   ATTN_SCORE_MOD_ALIBI:    S_ij = scale * <Q_i, K_j> + slope[hq] * (j - p)
+ *   ATTN_SCORE_MOD_REL_BIAS: S_ij = scale * <Q_i, K_j> + table[hq][clamp(j - p,
+ *                            -R, R) + R]
+ * score_mod, score_mod_params and score_mod_arg as for attn_fwd_score_mod
+ * (slopes [Hq] or table [Hq][2R + 1], fp32 device arrays, read only); the
+ * other arguments, the workspace and the errors as attn_decode_splitkv, plus
+ * INVALID_ARG for an unknown score_mod, missing params or R outside [0, 2^20].
+ */
+attn_status_t attn_decode_splitkv_score_mod(const void* q, const void* k_cache,
+                                            const void* v_cache, void* o, float* lse,
+                                            const int32_t* kv_lens, int B, int Hq, int Hkv,
+                                            int Lq, int Lk_max, int d, float scale,
+                                            int num_splits, int score_mod,
+                                            const float* score_mod_params, int score_mod_arg,
+                                            void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * attn_decode_paged — the split-KV decode of attn_decode_splitkv over a paged
  * KV cache (the paged block_table call of "FlexAttention 是什么，以及 DFlash2 之谜
  * 的完整侦破", section 4, experiment 1; PagedAttention through a logical-to-
@@ -342,6 +364,18 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
                                 int page_size, int pages_per_seq, int num_pages, int d,
                                 float scale, int num_splits, void* workspace, size_t ws_bytes,
                                 void* stream);
+
+/*
+ * attn_decode_paged_score_mod — attn_decode_paged with a score modifier, with
+ * the positions and arguments of attn_decode_splitkv_score_mod.
+ */
+attn_status_t attn_decode_paged_score_mod(const void* q, const void* k_pages, const void* v_pages,
+                                          const int32_t* block_table, void* o, float* lse,
+                                          const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
+                                          int page_size, int pages_per_seq, int num_pages, int d,
+                                          float scale, int num_splits, int score_mod,
+                                          const float* score_mod_params, int score_mod_arg,
+                                          void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * attn_decode_splitkv_noalloc — attn_decode_splitkv for callers that cannot

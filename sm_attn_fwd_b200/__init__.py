@@ -30,6 +30,7 @@ __all__ = [
     "attn_fwd_host", "attn_fwd_host_workspace_size",
     "attn_decode_num_splits", "SCORE_MOD_NONE", "SCORE_MOD_ALIBI", "SCORE_MOD_REL_BIAS",
     "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
+    "attn_decode_splitkv_score_mod", "attn_decode_paged_score_mod",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
     "EXPORTED_SYMBOLS",
 ]
@@ -55,6 +56,7 @@ EXPORTED_SYMBOLS = (
     "attn_bwd_workspace_size", "attn_bwd",
     "attn_decode_num_splits", "attn_decode_workspace_size",
     "attn_decode_splitkv", "attn_decode_paged", "attn_decode_splitkv_noalloc",
+    "attn_decode_splitkv_score_mod", "attn_decode_paged_score_mod",
     "attn_get_device_error", "attn_selftest_wait_timeout", "attn_status_string",
 )
 
@@ -118,6 +120,13 @@ def load_library():
         lib.attn_decode_paged.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
                                           i32, f32, i32, P, sz, P]
         lib.attn_decode_paged.restype = i32
+        lib.attn_decode_splitkv_score_mod.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                                      i32, f32, i32, i32, P, i32, P, sz, P]
+        lib.attn_decode_splitkv_score_mod.restype = i32
+        lib.attn_decode_paged_score_mod.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i32,
+                                                    i32, i32, i32, f32, i32, i32, P, i32, P, sz,
+                                                    P]
+        lib.attn_decode_paged_score_mod.restype = i32
         lib.attn_decode_splitkv_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i32,
                                                     i32, f32, i32, P]
         lib.attn_decode_splitkv_noalloc.restype = i32
@@ -383,6 +392,23 @@ def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, *, scale=None, num_splits=
     on the device.  ``workspace`` (uint8 CUDA tensor) is allocated here when
     not given.  Returns (o, lse).
     """
+    return _decode(q, k_cache, v_cache, kv_lens, scale, num_splits, workspace, o, lse, stream,
+                   None)
+
+
+def attn_decode_splitkv_score_mod(q, k_cache, v_cache, kv_lens, *, alibi_slopes=None,
+                                  rel_bias=None, scale=None, num_splits=0, workspace=None,
+                                  o=None, lse=None, stream=None):
+    """attn_decode_splitkv with a score modifier (see ``attn_decode_splitkv_score_mod``
+    in include/attn.h): ``alibi_slopes`` (fp32 CUDA tensor [Hq]) or ``rel_bias`` =
+    (table fp32 CUDA tensor [Hq, 2R + 1], R), with query row i of sequence b at
+    position kv_lens[b] - Lq + i.  Returns (o, lse)."""
+    mod = _score_mod_args(q.shape[1], alibi_slopes, rel_bias)
+    return _decode(q, k_cache, v_cache, kv_lens, scale, num_splits, workspace, o, lse, stream,
+                   mod)
+
+
+def _decode(q, k_cache, v_cache, kv_lens, scale, num_splits, workspace, o, lse, stream, mod):
     for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _check_bf16(name, t)
     if kv_lens.dtype != torch.int32 or not kv_lens.is_cuda or not kv_lens.is_contiguous():
@@ -398,12 +424,19 @@ def attn_decode_splitkv(q, k_cache, v_cache, kv_lens, *, scale=None, num_splits=
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    st = load_library().attn_decode_splitkv(
-        _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), _ptr(kv_lens), B, Hq, Hkv,
-        Lq, Lk_max, d, float(scale), int(num_splits), _ptr(workspace),
-        workspace.numel() * workspace.element_size(), _stream_handle(stream, q.device))
+    ws_bytes = workspace.numel() * workspace.element_size()
+    head = (_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse), _ptr(kv_lens), B, Hq, Hkv,
+            Lq, Lk_max, d, float(scale), int(num_splits))
+    tail = (_ptr(workspace), ws_bytes, _stream_handle(stream, q.device))
+    if mod is None:
+        name = "attn_decode_splitkv"
+        st = load_library().attn_decode_splitkv(*head, *tail)
+    else:
+        name = "attn_decode_splitkv_score_mod"
+        kind, params, arg = mod
+        st = load_library().attn_decode_splitkv_score_mod(*head, kind, _ptr(params), arg, *tail)
     if st != ATTN_OK:
-        raise AttnError(st, "attn_decode_splitkv")
+        raise AttnError(st, name)
     return o, lse
 
 
@@ -414,6 +447,22 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, *, scale=None, 
     q: [B, Hq, Lq, d]; k_pages/v_pages: [num_pages, Hkv, page_size, d] bf16;
     block_table: int32 [B, pages_per_seq]; kv_lens: int32 [B] (device).
     """
+    return _decode_paged(q, k_pages, v_pages, block_table, kv_lens, scale, num_splits, workspace,
+                         o, lse, stream, None)
+
+
+def attn_decode_paged_score_mod(q, k_pages, v_pages, block_table, kv_lens, *, alibi_slopes=None,
+                                rel_bias=None, scale=None, num_splits=0, workspace=None, o=None,
+                                lse=None, stream=None):
+    """attn_decode_paged with a score modifier, as ``attn_decode_splitkv_score_mod``
+    (see ``attn_decode_paged_score_mod`` in include/attn.h)."""
+    mod = _score_mod_args(q.shape[1], alibi_slopes, rel_bias)
+    return _decode_paged(q, k_pages, v_pages, block_table, kv_lens, scale, num_splits, workspace,
+                         o, lse, stream, mod)
+
+
+def _decode_paged(q, k_pages, v_pages, block_table, kv_lens, scale, num_splits, workspace, o,
+                  lse, stream, mod):
     for name, t in (("q", q), ("k_pages", k_pages), ("v_pages", v_pages)):
         _check_bf16(name, t)
     for name, t in (("block_table", block_table), ("kv_lens", kv_lens)):
@@ -431,13 +480,20 @@ def attn_decode_paged(q, k_pages, v_pages, block_table, kv_lens, *, scale=None, 
         o = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    st = load_library().attn_decode_paged(
-        _ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(o), _ptr(lse),
-        _ptr(kv_lens), B, Hq, Hkv, Lq, page_size, pages_per_seq, num_pages, d, float(scale),
-        int(num_splits), _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream_handle(stream, q.device))
+    head = (_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table), _ptr(o), _ptr(lse),
+            _ptr(kv_lens), B, Hq, Hkv, Lq, page_size, pages_per_seq, num_pages, d, float(scale),
+            int(num_splits))
+    tail = (_ptr(workspace), workspace.numel() * workspace.element_size(),
+            _stream_handle(stream, q.device))
+    if mod is None:
+        name = "attn_decode_paged"
+        st = load_library().attn_decode_paged(*head, *tail)
+    else:
+        name = "attn_decode_paged_score_mod"
+        kind, params, arg = mod
+        st = load_library().attn_decode_paged_score_mod(*head, kind, _ptr(params), arg, *tail)
     if st != ATTN_OK:
-        raise AttnError(st, "attn_decode_paged")
+        raise AttnError(st, name)
     return o, lse
 
 

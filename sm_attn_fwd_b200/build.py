@@ -19,7 +19,8 @@ LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libattn_b200.so")
 SOURCES = ["attn_api.cu", "attn_kernels.cu", "attn_prefill.cu", "attn_short.cu", "attn_noalloc.cu",
            "attn_backward.cu"]
-HEADERS = ["attn_params.h", "attn_bwd_params.h", "ptx.cuh", "host_once.h", "prefill_common.cuh"]
+HEADERS = ["attn_params.h", "attn_bwd_params.h", "ptx.cuh", "host_once.h", "prefill_common.cuh",
+           "softmax_row.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

@@ -351,7 +351,7 @@ struct ScoreMod {
   int rel_max = 0;
 };
 
-// Checks the score_mod arguments of attn_fwd_score_mod / attn_fwd_varlen_score_mod.
+// Checks the score_mod arguments of the *_score_mod entry points.
 static attn_status_t parse_score_mod(int kind, const float* params, int arg, ScoreMod* sm) {
   *sm = ScoreMod{};
   if (kind == ATTN_SCORE_MOD_NONE) return ATTN_OK;
@@ -825,7 +825,7 @@ struct PagedKv {
 attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cache, void* o,
                           float* lse, const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
                           int Lk_max, int d, float scale, int num_splits, void* workspace,
-                          size_t ws_bytes, void* stream, const PagedKv& pg) {
+                          size_t ws_bytes, void* stream, const PagedKv& pg, const ScoreMod& sm) {
   if (!q || !k_cache || !v_cache || !o || !lse || !kv_lens) return ATTN_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
       !aligned(lse, 4) || !aligned(kv_lens, 4))
@@ -863,6 +863,9 @@ attn_status_t decode_impl(const void* q, const void* k_cache, const void* v_cach
   p.chunk = pl.chunk;
   p.nsplit = pl.nsplit;
   p.row_tiles = pl.row_tiles;
+  p.alibi_slopes = sm.alibi_slopes;
+  p.rel_table = sm.rel_table;
+  p.rel_max = sm.rel_max;
   p.block_table = pg.block_table;
   p.page_size = pg.page_size;
   p.pages_per_seq = pg.pages_per_seq;
@@ -901,15 +904,32 @@ attn_status_t attn_decode_splitkv(const void* q, const void* k_cache, const void
                                   int Hkv, int Lq, int Lk_max, int d, float scale, int num_splits,
                                   void* workspace, size_t ws_bytes, void* stream) {
   return decode_impl(q, k_cache, v_cache, o, lse, kv_lens, B, Hq, Hkv, Lq, Lk_max, d, scale,
-                     num_splits, workspace, ws_bytes, stream, PagedKv{});
+                     num_splits, workspace, ws_bytes, stream, PagedKv{}, ScoreMod{});
 }
 
-attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
-                                const int32_t* block_table, void* o, float* lse,
-                                const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
-                                int page_size, int pages_per_seq, int num_pages, int d,
-                                float scale, int num_splits, void* workspace, size_t ws_bytes,
-                                void* stream) {
+attn_status_t attn_decode_splitkv_score_mod(const void* q, const void* k_cache,
+                                            const void* v_cache, void* o, float* lse,
+                                            const int32_t* kv_lens, int B, int Hq, int Hkv,
+                                            int Lq, int Lk_max, int d, float scale,
+                                            int num_splits, int score_mod,
+                                            const float* score_mod_params, int score_mod_arg,
+                                            void* workspace, size_t ws_bytes, void* stream) {
+  ScoreMod sm;
+  const attn_status_t st = parse_score_mod(score_mod, score_mod_params, score_mod_arg, &sm);
+  if (st != ATTN_OK) return st;
+  return decode_impl(q, k_cache, v_cache, o, lse, kv_lens, B, Hq, Hkv, Lq, Lk_max, d, scale,
+                     num_splits, workspace, ws_bytes, stream, PagedKv{}, sm);
+}
+
+}  // extern "C"
+
+namespace {
+
+attn_status_t paged_impl(const void* q, const void* k_pages, const void* v_pages,
+                         const int32_t* block_table, void* o, float* lse, const int32_t* kv_lens,
+                         int B, int Hq, int Hkv, int Lq, int page_size, int pages_per_seq,
+                         int num_pages, int d, float scale, int num_splits, void* workspace,
+                         size_t ws_bytes, void* stream, const ScoreMod& sm) {
   if (!block_table || !aligned(block_table, 4)) return ATTN_ERR_INVALID_ARG;
   if (page_size < 16 || page_size > (1 << 16) || (page_size & (page_size - 1)) != 0)
     return ATTN_ERR_INVALID_ARG;
@@ -923,7 +943,37 @@ attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* 
   pg.pages_per_seq = pages_per_seq;
   pg.num_pages = num_pages;
   return decode_impl(q, k_pages, v_pages, o, lse, kv_lens, B, Hq, Hkv, Lq, (int)lk, d, scale,
-                     num_splits, workspace, ws_bytes, stream, pg);
+                     num_splits, workspace, ws_bytes, stream, pg, sm);
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status_t attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                const int32_t* block_table, void* o, float* lse,
+                                const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
+                                int page_size, int pages_per_seq, int num_pages, int d,
+                                float scale, int num_splits, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  return paged_impl(q, k_pages, v_pages, block_table, o, lse, kv_lens, B, Hq, Hkv, Lq, page_size,
+                    pages_per_seq, num_pages, d, scale, num_splits, workspace, ws_bytes, stream,
+                    ScoreMod{});
+}
+
+attn_status_t attn_decode_paged_score_mod(const void* q, const void* k_pages, const void* v_pages,
+                                          const int32_t* block_table, void* o, float* lse,
+                                          const int32_t* kv_lens, int B, int Hq, int Hkv, int Lq,
+                                          int page_size, int pages_per_seq, int num_pages, int d,
+                                          float scale, int num_splits, int score_mod,
+                                          const float* score_mod_params, int score_mod_arg,
+                                          void* workspace, size_t ws_bytes, void* stream) {
+  ScoreMod sm;
+  const attn_status_t st = parse_score_mod(score_mod, score_mod_params, score_mod_arg, &sm);
+  if (st != ATTN_OK) return st;
+  return paged_impl(q, k_pages, v_pages, block_table, o, lse, kv_lens, B, Hq, Hkv, Lq, page_size,
+                    pages_per_seq, num_pages, d, scale, num_splits, workspace, ws_bytes, stream,
+                    sm);
 }
 
 attn_status_t attn_get_device_error(void* stream, int* raw_bits) {

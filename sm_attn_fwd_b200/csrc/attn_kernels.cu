@@ -11,16 +11,19 @@
 // [0, kv_lens[b]) of its sequence) and leaves a normalised partial output plus
 // its log-sum-exp for the combine kernel at the end of this file.
 //
-// B200 mapping (one CTA per SM, 192 threads):
+// B200 mapping (one CTA per SM, 256 threads):
 //   warp 0      TMA producer: Q once, then K and V tiles into a ring of stages
 //               (128-byte swizzled boxes, mbarrier transaction counts).
 //   warp 1      allocates tensor memory; lane 0 issues tcgen05.mma:
 //               S_j = Q K_j^T (both operands in shared memory, fp32 in TMEM),
 //               O  += P_j V_j (P from TMEM, V from shared memory, MN-major).
 //   warps 2..5  softmax: thread r owns query row r (its TMEM lane), loads S_j,
-//               masks partial tiles, updates m and l in base 2, rescales O only
-//               when the running max grew by more than 2^8, writes P_j as bf16
-//               over S_j in TMEM, and finally stores O / l and the LSE.
+//               masks partial tiles, adds the score modifier (ALiBi or a
+//               relative-position table, compile-time variants), updates m and
+//               l in base 2, rescales O only when the running max grew by more
+//               than 2^8, writes P_j as bf16 over S_j in TMEM, and finally
+//               stores O / l and the LSE.
+//   warps 6, 7  extra TMA copy warps for pages shorter than a key tile.
 // Tensor memory: S double buffer at columns [0,128) and [128,256), O at
 // [256, 256 + d).  Key tiles that the mask empties entirely are never loaded.
 // A paged cache whose pages are shorter than a key tile takes one TMA box per
@@ -36,6 +39,7 @@
 #include "attn_params.h"
 #include "host_once.h"
 #include "ptx.cuh"
+#include "softmax_row.cuh"
 
 namespace attn {
 
@@ -104,7 +108,9 @@ __device__ __forceinline__ uint64_t desc_v_mnmajor(uint32_t tile_saddr, int kk) 
 
 }  // namespace
 
-template <int D>
+// kMod: the score modifier (row::kModNone, kModAlibi or kModRelBias) with the
+// query row's absolute position p = kv_lens[b] - Lq + i.
+template <int D, int kMod>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_decode_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -394,6 +400,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     // every query row of the sequence sees the keys [0, kv_len); rows past the
     // tile's valid rows see none
     const long long row_hi = row_ok ? (long long)key_end - 1 : -1;
+    // score modifier: the row's query head and absolute position
+    const int row_flat = rt * kBlockM + (row_ok ? r : 0);  // (head in group, query) of the tile row
+    const int row_g = row_flat / p.Lq;
+    const long long row_pos = (long long)kv_len - p.Lq + (row_flat - row_g * p.Lq);
+    const int row_hq = hkv * p.group + row_g;
+    const float alibi2 =
+        kMod == row::kModAlibi ? __ldg(p.alibi_slopes + row_hq) * row::kLog2e : 0.0f;
+    const float* rel_row = kMod == row::kModRelBias
+                               ? p.rel_table + (long long)row_hq * (2 * p.rel_max + 1) + p.rel_max
+                               : nullptr;
+    const float c_s = kMod != row::kModNone ? 1.0f : c;  // scale still to apply to the scores
 
     float m_ref = -INFINITY;  // reference max (base-2 scaled units)
     float l = 0.0f;
@@ -410,14 +427,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_after();
 
       float s[kBlockN];
-      ptx::tmem_ld_row128(t_row + tmem_s(j), s);
+      row::tmem_ld_row128(t_row + tmem_s(j), s);
       if (!full) {
         // visible keys of this row inside the tile: [0, hi_rel]
         const int hi_rel = (int)max(-1LL, min((long long)kBlockN - 1, row_hi - k0));
 #pragma unroll
         for (int i = 0; i < kBlockN; ++i) s[i] = (i <= hi_rel) ? s[i] : -INFINITY;
       }
-      const float m_tile = ptx::row_max128(s) * c;
+      if constexpr (kMod != row::kModNone)
+        row::score_mod128<kMod>(s, c, (int)(k0 - row_pos), alibi2, rel_row, p.rel_max);
+      const float m_tile = ptx::row_max128(s) * c_s;
       const float m_new = fmaxf(m_ref, m_tile);
       const bool need = m_new > m_ref + kRescaleThreshold;
       const float alpha = need ? ptx::ex2(m_ref - m_new) : 1.0f;  // 0 when m_ref = -inf
@@ -446,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         // P over S: 64 columns of bf16 pairs
         uint32_t pk_lo[32], pk_hi[32];
-        l += ptx::exp2_pack128(s, c, m_use, pk_lo, pk_hi);
+        l += row::exp2_pack128(s, c_s, m_use, pk_lo, pk_hi);
         ptx::tmem_st32(t_row + tmem_s(j), pk_lo);
         ptx::tmem_st32(t_row + tmem_s(j) + 32, pk_hi);
       }
@@ -630,10 +649,11 @@ cudaError_t launch_selftest_wait(cudaStream_t stream) {
 }
 
 // ------------------------------------------------------------- launchers
-template <int D>
-cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const FwdParams& p, dim3 grid, cudaStream_t stream) {
-  auto kern = attn_decode_kernel<D>;
+template <int D, int kMod>
+cudaError_t launch_decode_kernel(const CUtensorMap& tq, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const FwdParams& p, dim3 grid,
+                                 cudaStream_t stream) {
+  auto kern = attn_decode_kernel<D, kMod>;
   constexpr int smem = Cfg<D>::kSmemAlloc;
   // The shared-memory opt-in is set once per device and context, normally by
   // a first call outside any stream capture that a later call may be part of.
@@ -644,6 +664,16 @@ cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   if (e != cudaSuccess) return e;
   kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_decode(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const FwdParams& p, dim3 grid, cudaStream_t stream) {
+  if (p.alibi_slopes)
+    return launch_decode_kernel<D, row::kModAlibi>(tq, tk, tv, p, grid, stream);
+  if (p.rel_table)
+    return launch_decode_kernel<D, row::kModRelBias>(tq, tk, tv, p, grid, stream);
+  return launch_decode_kernel<D, row::kModNone>(tq, tk, tv, p, grid, stream);
 }
 
 template <int D>

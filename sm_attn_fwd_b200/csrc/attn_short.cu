@@ -38,6 +38,7 @@
 #include "host_once.h"
 #include "prefill_common.cuh"
 #include "ptx.cuh"
+#include "softmax_row.cuh"
 
 namespace attn {
 
@@ -404,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         float s[kBlockN];
-        ptx::tmem_ld_row128(t_row + tmem_s(j), s);
+        row::tmem_ld_row128(t_row + tmem_s(j), s);
         if (!full) {
 #pragma unroll
           for (int i = 0; i < kBlockN; ++i)
@@ -439,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           // P over S: 64 columns of bf16 pairs
           uint32_t pk_lo[32], pk_hi[32];
-          l += ptx::exp2_pack128(s, c, m_use, pk_lo, pk_hi);
+          l += row::exp2_pack128(s, c, m_use, pk_lo, pk_hi);
           ptx::tmem_st32(t_row + tmem_s(j), pk_lo);
           ptx::tmem_st32(t_row + tmem_s(j) + 32, pk_hi);
         }

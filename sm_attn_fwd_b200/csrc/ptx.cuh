@@ -540,58 +540,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// The 128 fp32 columns [taddr, taddr + 128) of this thread's tensor-memory lane
-// (32x32b shape): all four 32-column loads in flight, one wait.
-__device__ __forceinline__ void tmem_ld_row128(uint32_t taddr, float (&s)[128]) {
-  uint32_t r0[32], r1[32], r2[32], r3[32];
-  tmem_ld32(taddr + 0, r0);
-  tmem_ld32(taddr + 32, r1);
-  tmem_ld32(taddr + 64, r2);
-  tmem_ld32(taddr + 96, r3);
-  tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    s[i] = __uint_as_float(r0[i]);
-    s[32 + i] = __uint_as_float(r1[i]);
-    s[64 + i] = __uint_as_float(r2[i]);
-    s[96 + i] = __uint_as_float(r3[i]);
-  }
-}
-
-// One row of P = 2^(s_i * c - m), i = 0..127, as 64 packed bf16 pairs (key 2i in
-// the low half; pairs 0..31 in lo, 32..63 in hi); returns the fp32 sum of the
-// unrounded values.  s * c - m is one packed fp32x2 FMA per pair; each pair's
-// exponentials are issued four pairs before the sum and packing that read them,
-// so the MUFU results are ready when needed; the sum runs in four packed chains.
-__device__ __forceinline__ float exp2_pack128(const float (&s)[128], float c, float m,
-                                              uint32_t (&lo)[32], uint32_t (&hi)[32]) {
-  constexpr int kAhead = 4;
-  float e0[kAhead], e1[kAhead];
-  float sum8[8];
-#pragma unroll
-  for (int k = 0; k < 8; ++k) sum8[k] = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 64 + kAhead; ++i) {
-    if (i >= kAhead) {
-      const int j = i - kAhead;
-      const float p0 = e0[j % kAhead], p1 = e1[j % kAhead];
-      add2_acc(sum8[(j & 3) * 2], sum8[(j & 3) * 2 + 1], p0, p1);
-      const uint32_t packed = pack_bf16x2(p0, p1);
-      if (j < 32) lo[j] = packed;
-      else hi[j - 32] = packed;
-    }
-    if (i < 64) {
-      float a0, a1;
-      fma2_bc(a0, a1, s[2 * i], s[2 * i + 1], c, -m);
-      e0[i % kAhead] = ex2(a0);
-      e1[i % kAhead] = ex2(a1);
-    }
-  }
-#pragma unroll
-  for (int k = 0; k < 4; ++k) sum8[k] += sum8[k + 4];
-  return (sum8[0] + sum8[1]) + (sum8[2] + sum8[3]);
-}
-
 // --------------------------------------------------- UMMA descriptors
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading and
 // stride byte offsets in 16-byte units, version 1, 128-byte swizzle.

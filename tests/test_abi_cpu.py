@@ -232,3 +232,26 @@ def test_binding_checks_tensors_before_calling_the_library():
     lse = torch.zeros(1, 2, 8)
     with pytest.raises(ValueError, match="CUDA"):
         ab.attn_bwd(q4, q4, q4, q4, lse, q4)
+
+
+def test_decode_score_mod_rejects_on_host():
+    lib = ab.load_library()
+    #       q  k  v  o  lse kv B  Hq Hkv Lq Lk    d    scale  ns
+    head = [A, A, A, A, A, A, 2, 16, 2, 1, 1000, 128, 0.125, 0]
+    ws = ctypes.c_void_p(0x100000)
+    need = lib.attn_decode_workspace_size(2, 16, 2, 1, 1000, 128, 0)
+    tail = [ws, need, None]
+    call = lib.attn_decode_splitkv_score_mod
+    assert call(*head, 7, A, 0, *tail) == ab.ATTN_ERR_INVALID_ARG          # unknown kind
+    assert call(*head, 1, None, 0, *tail) == ab.ATTN_ERR_INVALID_ARG       # no slopes
+    assert call(*head, 2, A, -1, *tail) == ab.ATTN_ERR_INVALID_ARG         # R < 0
+    assert call(*head, 2, A, (1 << 20) + 1, *tail) == ab.ATTN_ERR_INVALID_ARG
+    assert call(*head, 1, A, 0, ws, need - 256, None) == ab.ATTN_ERR_WORKSPACE
+    #        q  k  v  table o  lse kv B  Hq Hkv Lq P    pps np   d    scale  ns
+    phead = [A, A, A, A, A, A, A, 2, 16, 2, 1, 16, 8, 16, 128, 0.125, 0]
+    pcall = lib.attn_decode_paged_score_mod
+    assert pcall(*phead, 9, A, 0, *tail) == ab.ATTN_ERR_INVALID_ARG
+    assert pcall(*phead, 2, None, 3, *tail) == ab.ATTN_ERR_INVALID_ARG
+    bad_page = list(phead)
+    bad_page[11] = 24                                                     # not a power of two
+    assert pcall(*bad_page, 1, A, 0, *tail) == ab.ATTN_ERR_INVALID_ARG

@@ -163,3 +163,89 @@ def test_alibi_bench_workload_sampled_rows():
                              rows=rows, alibi_slopes=sl.double().numpy())
     idx = torch.from_numpy(rows).cuda()
     compare(o.reshape(-1, cfg.d)[idx], lse.reshape(-1)[idx], ro, rl, "alibi bench workload")
+
+
+# ---------------------------------------------------------------- decode
+DECODE_CASES = [
+    # seed, B, Hq, Hkv, Lq, Lk_max, d, (lo, hi), num_splits, kind
+    (31, 2, 8, 1, 1, 300, 128, (1, 300), 0, "alibi"),
+    (32, 3, 16, 2, 16, 1000, 128, (1, 1000), 3, "alibi"),
+    (33, 2, 4, 4, 3, 513, 64, (1, 513), 5, "rel"),
+    (34, 2, 32, 2, 16, 640, 128, (100, 640), 2, "rel"),   # two row tiles per kv head
+    (35, 1, 64, 8, 16, 2048, 128, (2048, 2048), 4, "alibi"),
+    (36, 4, 8, 8, 1, 129, 64, (1, 129), 0, "rel"),
+]
+
+
+def _mod_args(kind, Hq, seed):
+    """(device kwargs for the binding, oracle kwargs) of one score modifier."""
+    if kind == "alibi":
+        sl = slopes_for(Hq)
+        return dict(alibi_slopes=sl.cuda()), dict(alibi_slopes=sl.double().numpy())
+    R = 37
+    table = torch.randn(Hq, 2 * R + 1, generator=torch.Generator().manual_seed(seed))
+    return (dict(rel_bias=(table.cuda(), R)),
+            dict(rel_bias=(table.double().numpy(), R)))
+
+
+@pytest.mark.parametrize("case", DECODE_CASES,
+                         ids=lambda c: f"s{c[0]}_{c[9]}_lq{c[4]}_lk{c[5]}_d{c[6]}")
+def test_decode_score_mod_matches_oracle(case):
+    """Split-KV decode with ALiBi or the relative-position table, query row i of
+    sequence b at p = kv_lens[b] - Lq + i; K/V past kv_lens are NaN."""
+    seed, B, Hq, Hkv, Lq, Lk, d, rng, ns, kind = case
+    q, k, v, _, kv = random_case(seed, B, Hq, Hkv, Lq, Lk, d, kv_len_range=rng)
+    kp, vp = k.clone(), v.clone()
+    for b, L in enumerate(kv.tolist()):
+        kp[b, :, L:] = float("nan")
+        vp[b, :, L:] = float("nan")
+    dev_kw, ora_kw = _mod_args(kind, Hq, seed)
+    qd, kd, vd, kl = to_dev(q, kp, vp, kv)
+    o, lse = ab.attn_decode_splitkv_score_mod(qd, kd, vd, kl, num_splits=ns, **dev_kw)
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    ro, rl = oracle.attn_fwd(q, k, v, kv_lens=kv, **ora_kw)
+    compare(o, lse, ro, rl, str(case))
+
+
+@pytest.mark.parametrize("P,kind", [(128, "alibi"), (16, "rel")])
+def test_paged_decode_score_mod_equals_contiguous(P, kind):
+    """Identity page table: the paged and the contiguous score-modifier calls agree
+    to the bit."""
+    B, Hq, Hkv, Lq, d = 2, 16, 2, 4, 128
+    pps = 1024 // P
+    q, k, v, _, _ = random_case(41, B, Hq, Hkv, Lq, pps * P, d)
+    kv = torch.tensor([700, 1024], dtype=torch.int32)
+    kp = k.view(B, Hkv, pps, P, d).permute(0, 2, 1, 3, 4).reshape(B * pps, Hkv, P, d).contiguous()
+    vp = v.view(B, Hkv, pps, P, d).permute(0, 2, 1, 3, 4).reshape(B * pps, Hkv, P, d).contiguous()
+    table = torch.arange(B * pps, dtype=torch.int32).view(B, pps)
+    dev_kw, _ = _mod_args(kind, Hq, 42)
+    qd, kd, vd, kpd, vpd, td, kvd = to_dev(q, k, v, kp, vp, table, kv)
+    o1, l1 = ab.attn_decode_splitkv_score_mod(qd, kd, vd, kvd, **dev_kw)
+    o2, l2 = ab.attn_decode_paged_score_mod(qd, kpd, vpd, td, kvd, **dev_kw)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_decode_alibi_full_size_sampled():
+    """The Lq = 16 decode workload (B = 64, Hq = 64, Hkv = 8, kv_lens up to 32K,
+    d = 128) with ALiBi slopes: 6 whole sequences (every head and query) against
+    the oracle; biases reach slope * 32K."""
+    from workloads import DECODE_LQ16, make_inputs
+    cfg = DECODE_LQ16
+    inp = make_inputs(cfg, device="cuda")
+    sl = slopes_for(cfg.Hq)
+    o, lse = ab.attn_decode_splitkv_score_mod(inp.q, inp.k, inp.v, inp.kv_lens,
+                                              alibi_slopes=sl.cuda(), scale=cfg.softmax_scale)
+    torch.cuda.synchronize()
+    st, bits = ab.attn_get_device_error()
+    assert st == ab.ATTN_OK, (st, bits)
+    kv_host = inp.kv_lens.cpu()
+    for b in np.random.default_rng(3).choice(cfg.B, 6, replace=False).tolist():
+        L = int(kv_host[b])
+        kvb = torch.tensor([L], dtype=torch.int32)
+        ro, rl = oracle.attn_fwd(inp.q[b:b + 1].cpu(), inp.k[b:b + 1, :, :L].cpu(),
+                                 inp.v[b:b + 1, :, :L].cpu(), scale=cfg.softmax_scale,
+                                 kv_lens=kvb, alibi_slopes=sl.double().numpy())
+        compare(o[b:b + 1], lse[b:b + 1], ro, rl, f"decode alibi b={b}")

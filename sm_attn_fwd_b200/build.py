@@ -38,7 +38,8 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def source_digest(files=("attn_prefill.cu", "prefill_common.cuh", "ptx.cuh", "attn_params.h")) -> str:
+def source_digest(files=("attn_prefill.cu", "prefill_common.cuh", "ptx.cuh", "attn_params.h",
+                         "softmax_row.cuh")) -> str:
     """Digest of one kernel's sources and the flags (identifies a profiled
     build); by default the prefill kernel's."""
     h = hashlib.sha256()

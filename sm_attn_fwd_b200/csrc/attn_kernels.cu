@@ -271,6 +271,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!small_pages) return lane < C::kAtoms ? page_z(t * kBlockN) : -1;
         return lane < mine ? page_z(t * kBlockN + (item / C::kAtoms) * p.page_size) : -1;
       };
+      // K/V tiles are read once: evict them from L2 first, so that the split
+      // partials this launch writes stay there for the combine that reads them
+      const uint64_t kv_policy = ptx::l2_policy_evict_first();
       auto load_kv = [&](uint8_t* dst, const CUtensorMap* tm, uint64_t* bar, int k0, int pz) {
         if (!small_pages) {
           if (lane == 0) ptx::mbar_arrive_expect_tx(bar, kTx);
@@ -278,15 +281,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane < C::kAtoms) {
             const int y = p.block_table == nullptr ? k0 : k0 % p.page_size;
             const int z = p.block_table == nullptr ? kv_z : pz;
-            ptx::tma_load_3d(dst + lane * C::kAtomBytes, tm, bar, lane * 64, y, z);
+            ptx::tma_load_3d_hint(dst + lane * C::kAtomBytes, tm, bar, lane * 64, y, z,
+                                  kv_policy);
           }
         } else {
           if (lane == 0) ptx::mbar_arrive_expect_tx(bar, (uint32_t)(mine * p.page_size * 128));
           __syncwarp();
           if (lane < mine) {
             const int sub = item / C::kAtoms, a = item % C::kAtoms;
-            ptx::tma_load_3d(dst + a * C::kAtomBytes + sub * p.page_size * 128, tm, bar, a * 64,
-                             0, pz);
+            ptx::tma_load_3d_hint(dst + a * C::kAtomBytes + sub * p.page_size * 128, tm, bar,
+                                  a * 64, 0, pz, kv_policy);
           }
         }
       };

@@ -38,6 +38,7 @@
 #include "host_once.h"
 #include "prefill_common.cuh"
 #include "ptx.cuh"
+#include "softmax_row.cuh"
 
 namespace attn {
 namespace {
@@ -57,7 +58,9 @@ constexpr int kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
-enum : int { kModNone = 0, kModAlibi = 1, kModRelBias = 2 };
+using row::kModAlibi;
+using row::kModNone;
+using row::kModRelBias;
 
 using Sched = prefill::Sched<128>;
 
@@ -671,47 +674,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             sv[i] = ((word >> (i & 31)) & 1u) ? sv[i] : -INFINITY;
           }
         }
-        if constexpr (kMod == kModRelBias) {
-          // scores to the base-2 domain with the table's bias:
-          // s*c + table[clamp(j - p, -R, R)]*log2(e); masked scores stay -inf.
-          // A tile whose keys all lie R or more from the row on one side takes
-          // one clamped value; only tiles within R of the row look keys up.
-          const int R = p.rel_max;
-          const int dj0 = k0 - (int)row_pos;  // j - p at the tile's first key
-          if (dj0 + 127 <= -R || dj0 >= R) {
-            const float bias = __ldg(rel_row + (dj0 >= R ? R : -R)) * kLog2e;
-#pragma unroll
-            for (int i = 0; i < 64; ++i)
-              ptx::fma2_bc(sv[2 * i], sv[2 * i + 1], sv[2 * i], sv[2 * i + 1], c, bias);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 128; ++i) {
-              const int delta = min(max(dj0 + i, -R), R);
-              sv[i] = fmaf(__ldg(rel_row + delta), kLog2e, sv[i] * c);
-            }
-          }
-        }
-        if constexpr (kMod == kModAlibi) {
-          // scores to the base-2 domain with the bias: s*c + slope*log2(e)*(j - p);
-          // masked scores stay -inf.  The max and the exponentials below then
-          // use a scale of 1.
-          // The bias of key pair i (keys 2i, 2i+1) comes from one of eight chains
-          // that step 16 keys at a time: one packed add and one packed FMA per pair.
-          const float base = alibi2 * (float)(k0 - row_pos);
-          const float step = alibi2 * 16.0f;
-          float b0[8], b1[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            b0[k] = fmaf(alibi2, (float)(2 * k), base);
-            b1[k] = fmaf(alibi2, (float)(2 * k + 1), base);
-          }
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int k = i & 7;
-            ptx::fma2_bv(sv[2 * i], sv[2 * i + 1], sv[2 * i], sv[2 * i + 1], c, b0[k], b1[k]);
-            if (i + 8 < 64) ptx::add2_acc(b0[k], b1[k], step, step);
-          }
-        }
+        // scores to the base-2 domain with the score modifier (masked scores stay
+        // -inf); the max and the exponentials below then use a scale of 1
+        if constexpr (kMod != kModNone)
+          row::score_mod128<kMod>(sv, c, (int)(k0 - row_pos), alibi2, rel_row, p.rel_max);
         // row max: sixteen independent chains of two-input max, then a tree
         float mx16[16];
 #pragma unroll

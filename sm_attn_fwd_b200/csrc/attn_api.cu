@@ -245,14 +245,14 @@ bool plan_splits(int B, int Hq, int Hkv, int Lq, int Lk_max, int d, int num_spli
   if (num_splits > 0) {
     splits = num_splits < max_splits ? num_splits : max_splits;
   } else {
-    // At least two waves of CTAs over the SMs, and chunks of at most 8192 keys
+    // At least two waves of CTAs over the SMs, and chunks of at most 12288 keys
     // so that ragged per-sequence lengths balance across the grid.  Shorter
     // chunks cost more than they balance: each split CTA pays a fixed start
     // (Q load, pipeline fill) and end (epilogue, its partial rows written here
-    // and read back by the combine), about 8 % of a 4096-key chunk.
+    // and read back by the combine, 512 bytes per query row and split).
     const long long units = (long long)B * Hkv * row_tiles;
     long long want = ceil_div(2LL * num_sms(), units);
-    const long long by_len = ceil_div(Lk_max, 8192);
+    const long long by_len = ceil_div(Lk_max, 12288);
     if (by_len > want) want = by_len;
     splits = want < max_splits ? want : max_splits;
   }

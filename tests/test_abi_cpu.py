@@ -90,8 +90,8 @@ def test_decode_split_plan_and_workspace_arithmetic():
     assert (n, chunk.value) == (8, 128)           # capped at ceil(1000 / 128)
     # library choice: chunks never exceed 8192 keys and cover Lk_max
     n = lib.attn_decode_num_splits(64, 64, 8, 1, 32768, 128, 0, ctypes.byref(chunk))
-    assert chunk.value <= 8192 and chunk.value % 128 == 0 and n * chunk.value >= 32768
-    assert (n, chunk.value) == (4, 8192)
+    assert chunk.value <= 12288 and chunk.value % 128 == 0 and n * chunk.value >= 32768
+    assert (n, chunk.value) == (3, 11008)
     # few (b, kv head) units: at least two waves of CTAs over the SMs
     n = lib.attn_decode_num_splits(1, 8, 1, 1, 32768, 128, 0, ctypes.byref(chunk))
     assert n * 1 >= 2 * 148 or chunk.value == 128

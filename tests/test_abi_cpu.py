@@ -255,3 +255,19 @@ def test_decode_score_mod_rejects_on_host():
     bad_page = list(phead)
     bad_page[11] = 24                                                     # not a power of two
     assert pcall(*bad_page, 1, A, 0, *tail) == ab.ATTN_ERR_INVALID_ARG
+
+
+def test_decode_score_mod_binding_rejects_bad_modifiers():
+    """The binding checks the modifier tensors before anything reaches the device."""
+    import torch
+    q = torch.zeros(1, 8, 1, 64, dtype=torch.bfloat16)
+    k = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16)
+    kv = torch.tensor([128], dtype=torch.int32)
+    slopes = torch.ones(8)
+    table = torch.zeros(8, 5)
+    with pytest.raises(ValueError):   # both modifiers
+        ab.attn_decode_splitkv_score_mod(q, k, k, kv, alibi_slopes=slopes, rel_bias=(table, 2))
+    with pytest.raises(ValueError):   # slopes not on the device
+        ab.attn_decode_splitkv_score_mod(q, k, k, kv, alibi_slopes=slopes)
+    with pytest.raises(ValueError):   # table not [Hq, 2R + 1] on the device
+        ab.attn_decode_paged_score_mod(q, k, k, kv.view(1, 1), kv, rel_bias=(table, 3))

@@ -363,6 +363,28 @@ def run_decode(cfg, timer, steps, warmup, stream):
     return inp, ms, decode_bytes(cfg, kv), (nsplit, chunk)
 
 
+def run_decode_alibi(cfg, timer, steps, warmup, stream):
+    """The decode workload with the ALiBi score_mod (slopes 2^(-8 (h+1) / Hq)), query row
+    i of sequence b at position kv_lens[b] - Lq + i."""
+    import sm_attn_fwd_b200 as ab
+    inp = make_inputs(cfg, device="cuda")
+    slopes = torch.tensor([2.0 ** (-8.0 * (h + 1) / cfg.Hq) for h in range(cfg.Hq)],
+                          dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    ws = torch.empty(ab.attn_decode_workspace_size(cfg.B, cfg.Hq, cfg.Hkv, cfg.Lq, cfg.Lk, cfg.d),
+                     dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(inp.q)
+    lse = torch.empty(cfg.B, cfg.Hq, cfg.Lq, dtype=torch.float32, device="cuda")
+    fn = lambda: ab.attn_decode_splitkv_score_mod(  # noqa: E731
+        inp.q, inp.k, inp.v, inp.kv_lens, alibi_slopes=slopes, scale=cfg.softmax_scale,
+        workspace=ws, o=o, lse=lse, stream=stream)
+    ms = timer.time(fn, steps, warmup)
+    st, bits = ab.attn_get_device_error(stream)
+    if st != ab.ATTN_OK:
+        raise RuntimeError(f"device error after {cfg.name} with ALiBi: {st} {bits}")
+    return ms, decode_bytes(cfg, inp.kv_lens.cpu().numpy())
+
+
 def run_decode_paged(cfg, page_size, timer, steps, warmup, stream):
     """The decode workload with its cache moved into a shuffled page pool
     [num_pages, Hkv, page_size, d] addressed through a block table."""
@@ -634,6 +656,12 @@ def main():
                                       "frac_of_8TBs_nominal": gbs / 8000.0,
                                       "algorithmic_bytes": nb, "splits": plan[0],
                                       "chunk_keys": plan[1]}
+            ms8, nb8 = run_decode_alibi(DECODE_LQ1, timer, max(5, args.steps // 10), 3, stream)
+            med = statistics.median(ms8)
+            gbs = nb8 / (med * 1e6)
+            workloads[DECODE_LQ1.name + "_alibi"] = {
+                "ms_median": med, "ms_min": min(ms8), "GB/s": gbs,
+                "frac_of_hbm": gbs / peaks["hbm_gbs"], "algorithmic_bytes": nb8}
             for psz in (128, 16):
                 ms4, nb4 = run_decode_paged(DECODE_LQ1, psz, timer, max(5, args.steps // 10), 3,
                                             stream)

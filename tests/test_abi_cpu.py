@@ -271,3 +271,19 @@ def test_decode_score_mod_binding_rejects_bad_modifiers():
         ab.attn_decode_splitkv_score_mod(q, k, k, kv, alibi_slopes=slopes)
     with pytest.raises(ValueError):   # table not [Hq, 2R + 1] on the device
         ab.attn_decode_paged_score_mod(q, k, k, kv.view(1, 1), kv, rel_bias=(table, 3))
+
+
+def test_decode_split_plan_rule():
+    """Without num_splits: at least two waves of CTAs over the SMs, and chunks of
+    at most 12288 keys (a multiple of 128) covering Lk_max."""
+    lib = ab.load_library()
+    chunk = ctypes.c_int(0)
+    # many (b, kv head) units: the chunk cap alone decides
+    for lk, want in ((12288, 1), (12289, 2), (32768, 3), (65536, 6), (131072, 11)):
+        n = lib.attn_decode_num_splits(64, 64, 8, 1, lk, 128, 0, ctypes.byref(chunk))
+        assert n == want, (lk, n)
+        assert chunk.value % 128 == 0 and chunk.value <= 12288 and n * chunk.value >= lk
+        assert (n - 1) * chunk.value < lk  # no empty split
+    # an explicit count is taken as given (up to one split per key tile)
+    assert lib.attn_decode_num_splits(64, 64, 8, 1, 32768, 128, 5, None) == 5
+    assert lib.attn_decode_num_splits(1, 8, 1, 1, 300, 128, 50, None) == 3

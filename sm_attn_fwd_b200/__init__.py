@@ -26,7 +26,8 @@ __all__ = [
     "AttnError", "ATTN_OK", "ATTN_ERR_INVALID_ARG", "ATTN_ERR_UNSUPPORTED",
     "ATTN_ERR_WORKSPACE", "ATTN_ERR_CUDA", "ATTN_ERR_TIMEOUT",
     "MASK_NONE", "MASK_CAUSAL", "MASK_DRAFT_BLOCK", "lib_path", "load_library",
-    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_bwd", "attn_decode_splitkv",
+    "attn_fwd", "attn_fwd_score_mod", "attn_fwd_varlen", "attn_fwd_varlen_score_mod",
+    "attn_bwd", "attn_bwd_workspace_size", "attn_decode_splitkv",
     "attn_fwd_host", "attn_fwd_host_workspace_size",
     "attn_decode_num_splits", "SCORE_MOD_NONE", "SCORE_MOD_ALIBI", "SCORE_MOD_REL_BIAS",
     "attn_decode_workspace_size", "attn_decode_paged", "attn_decode_splitkv_noalloc",
@@ -293,6 +294,14 @@ def attn_fwd_score_mod(q, k, v, *, alibi_slopes=None, rel_bias=None, scale=None,
     return o, lse
 
 
+def attn_bwd_workspace_size(B, Hq, Lq, d) -> int:
+    """Bytes of workspace attn_bwd needs (see ``attn_bwd_workspace_size`` in include/attn.h)."""
+    n = load_library().attn_bwd_workspace_size(B, Hq, Lq, d)
+    if n == 0:
+        raise AttnError(ATTN_ERR_INVALID_ARG, "attn_bwd_workspace_size")
+    return int(n)
+
+
 def attn_bwd(q, k, v, o, lse, dout, *, scale=None, mask="none", window=(-1, -1), draft_block=1,
              doc_ids=None, workspace=None, dq=None, dk=None, dv=None, stream=None):
     """Gradients of attn_fwd (see ``attn_bwd`` in include/attn.h): returns (dq, dk, dv).
@@ -375,6 +384,17 @@ def attn_decode_num_splits(B, Hq, Hkv, Lq, Lk_max, d, num_splits=0):
     if n < 0:
         raise AttnError(ATTN_ERR_INVALID_ARG, "attn_decode_num_splits")
     return int(n), int(chunk.value)
+
+
+def attn_fwd_varlen_score_mod(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, *,
+                              alibi_slopes=None, rel_bias=None, **kw):
+    """attn_fwd_varlen with a score modifier (see ``attn_fwd_varlen_score_mod`` in
+    include/attn.h): ``alibi_slopes`` or ``rel_bias`` as in ``attn_fwd_score_mod``,
+    each sequence's own positions; the other arguments as attn_fwd_varlen."""
+    if alibi_slopes is None and rel_bias is None:
+        raise ValueError("give alibi_slopes or rel_bias")
+    return attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q,
+                           alibi_slopes=alibi_slopes, rel_bias=rel_bias, **kw)
 
 
 def attn_decode_workspace_size(B, Hq, Hkv, Lq, Lk_max, d, num_splits=0) -> int:

@@ -24,6 +24,13 @@ def test_header_declares_the_documented_entry_points():
     assert set(declared_functions()) == set(ab.EXPORTED_SYMBOLS)
 
 
+def test_binding_has_every_entry_point_under_its_name():
+    """The Python binding offers each C entry point under the same name."""
+    missing = [name for name in declared_functions()
+               if not callable(getattr(ab, name, None)) or name not in ab.__all__]
+    assert not missing, missing
+
+
 def test_library_exports_every_declared_symbol():
     lib = ab.load_library()
     for name in declared_functions():
